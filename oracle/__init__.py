@@ -1,0 +1,217 @@
+"""CPU oracle for patch-restricted self-attention (float64).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, by ``__graft_entry__.smoke``
+and by the benchmark's CPU-baseline leg. The library's compute path never
+imports it, and it shares no code with the CUDA sources.
+
+Two independent formulations of the same definition:
+
+* :func:`npa_attention` / :func:`pcpp_attention` call the C gather oracle
+  (``npa_oracle.c``): per query, build the key set from the definition, gather,
+  softmax in double. OpenMP over queries only.
+* :func:`dense_attention` builds the full ``[N, N+G]`` membership mask from a
+  coordinate predicate and applies a masked softmax with NumPy, float64. It is
+  only meant for small grids (up to ~64x64 tokens).
+
+Definitions followed (see ``npa_oracle.c`` for the readings taken where the
+pages are silent):
+  * NPA: ScaleDiff (atlas.scime.ai summary), "Approach": non-overlapping query
+    patches, each attending to an overlapping K/V neighbourhood (patch grown by
+    a margin, clipped to the grid).
+  * PCPP: Partially Conditioned Patch Parallelism (pith.science review), "What
+    carries the argument" / "Core claim": a strip attends to itself plus the
+    p-fraction of each adjacent strip's height next to it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "lib", "npa_key_set", "pcpp_key_set", "pcpp_neighbor_rows", "npa_attention",
+    "pcpp_attention", "pair_count", "num_threads", "dense_mask", "dense_attention",
+    "bf16_to_f64",
+]
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        u16p = ctypes.c_void_p
+        L.oracle_npa_key_set.argtypes = [ctypes.c_int] * 5 + [i32p]
+        L.oracle_npa_key_set.restype = ctypes.c_int
+        L.oracle_pcpp_key_set.argtypes = [ctypes.c_int] * 3 + [ctypes.c_double, ctypes.c_int, i32p]
+        L.oracle_pcpp_key_set.restype = ctypes.c_int
+        L.oracle_pcpp_neighbor_rows.argtypes = [ctypes.c_int, ctypes.c_double]
+        L.oracle_pcpp_neighbor_rows.restype = ctypes.c_int
+        common = [u16p] * 5 + [ctypes.c_void_p] + [ctypes.c_int] * 5
+        L.oracle_npa_attention.argtypes = common + [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_void_p, ctypes.c_long]
+        L.oracle_npa_attention.restype = ctypes.c_int
+        L.oracle_pcpp_attention.argtypes = common + [ctypes.c_int, ctypes.c_double, ctypes.c_int,
+                                                     ctypes.c_void_p, ctypes.c_long]
+        L.oracle_pcpp_attention.restype = ctypes.c_int
+        L.oracle_pair_count.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
+        L.oracle_pair_count.restype = ctypes.c_longlong
+        L.oracle_num_threads.argtypes = []
+        L.oracle_num_threads.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bit patterns to float64."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def npa_key_set(H: int, W: int, P: int, m: int, t: int) -> np.ndarray:
+    buf = np.empty(H * W, dtype=np.int32)
+    n = lib().oracle_npa_key_set(H, W, P, m, t, buf.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    if n < 0:
+        raise ValueError("bad NPA key-set arguments")
+    return buf[:n].copy()
+
+
+def pcpp_key_set(H: int, W: int, n_strips: int, p: float, t: int) -> np.ndarray:
+    buf = np.empty(H * W, dtype=np.int32)
+    n = lib().oracle_pcpp_key_set(H, W, n_strips, float(p), t,
+                                  buf.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    if n < 0:
+        raise ValueError("bad PCPP key-set arguments")
+    return buf[:n].copy()
+
+
+def pcpp_neighbor_rows(strip_rows: int, p: float) -> int:
+    return int(lib().oracle_pcpp_neighbor_rows(strip_rows, float(p)))
+
+
+def pair_count(geometry: str, H: int, W: int, *, patch: int = 0, margin: int = 0,
+               n_strips: int = 0, p: float = 0.0, G: int = 0) -> int:
+    """Sum over all queries of one (b, h) of the key-set size (image + global)."""
+    g = 0 if geometry == "npa" else 1
+    a = patch if g == 0 else n_strips
+    b = margin if g == 0 else 0
+    n = lib().oracle_pair_count(g, H, W, a, b, float(p), G)
+    if n < 0:
+        raise ValueError("bad geometry")
+    return int(n)
+
+
+def _u16(x: Optional[np.ndarray]):
+    if x is None:
+        return None, None
+    a = np.ascontiguousarray(x, dtype=np.uint16)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _call(fn, geometry_args, q, k, v, gk, gv, B, heads, H, W, d, G, queries):
+    q, qp = _u16(q)
+    k, kp = _u16(k)
+    v, vp = _u16(v)
+    gk, gkp = _u16(gk)
+    gv, gvp = _u16(gv)
+    if queries is None:
+        out = np.empty((B, heads, H * W, d), dtype=np.float64)
+        qs_p, nq = None, 0
+    else:
+        qs = np.ascontiguousarray(np.asarray(queries, dtype=np.int32).reshape(-1, 3))
+        out = np.empty((qs.shape[0], d), dtype=np.float64)
+        qs_p, nq = qs.ctypes.data_as(ctypes.c_void_p), qs.shape[0]
+    rc = fn(qp, kp, vp, gkp, gvp, out.ctypes.data_as(ctypes.c_void_p), B, heads, H, W, d,
+            *geometry_args, G, qs_p, nq)
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return out
+
+
+def npa_attention(q, k, v, *, B, heads, H, W, d, patch, margin, gk=None, gv=None, G=0,
+                  queries: Optional[Sequence] = None) -> np.ndarray:
+    """NPA attention in float64. ``queries``: optional (n, 3) array of (b, h, t)."""
+    return _call(lib().oracle_npa_attention, (patch, margin), q, k, v, gk, gv, B, heads, H, W, d,
+                 G, queries)
+
+
+def pcpp_attention(q, k, v, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None, G=0,
+                   queries: Optional[Sequence] = None) -> np.ndarray:
+    """PCPP attention in float64. ``queries``: optional (n, 3) array of (b, h, t)."""
+    return _call(lib().oracle_pcpp_attention, (n_strips, float(p)), q, k, v, gk, gv, B, heads, H,
+                 W, d, G, queries)
+
+
+# ---------------------------------------------------------------------------
+# Dense formulation: a membership predicate over coordinates, then a masked
+# softmax over the full key axis.
+# ---------------------------------------------------------------------------
+
+def dense_mask(geometry: str, H: int, W: int, *, patch: int = 0, margin: int = 0,
+               n_strips: int = 0, p: float = 0.0, G: int = 0) -> np.ndarray:
+    """Boolean ``[N, N+G]``: entry (t, j) is True when query t may attend key j.
+
+    NPA: key (r', c') is visible to query (r, c) when r' lies within ``margin``
+    rows of the query's patch row span and c' within ``margin`` columns of its
+    column span (the grid bounds clip automatically). PCPP: key row r' is
+    visible to a query in strip i when it lies in strip i, or in strip i-1 at
+    most ``r`` rows above strip i's first row, or in strip i+1 at most ``r``
+    rows below its last row.
+    """
+    N = H * W
+    rows = np.arange(N) // W
+    cols = np.arange(N) % W
+    if geometry == "npa":
+        P, m = patch, margin
+        pr0 = (rows // P) * P
+        pr1 = np.minimum(pr0 + P, H)
+        pc0 = (cols // P) * P
+        pc1 = np.minimum(pc0 + P, W)
+        ok_r = (rows[None, :] >= (pr0 - m)[:, None]) & (rows[None, :] < (pr1 + m)[:, None])
+        ok_c = (cols[None, :] >= (pc0 - m)[:, None]) & (cols[None, :] < (pc1 + m)[:, None])
+        img = ok_r & ok_c
+    elif geometry == "pcpp":
+        s = H // n_strips
+        r = pcpp_neighbor_rows(s, p)
+        qi = rows // s
+        ki = rows // s
+        dist_above = (qi[:, None] * s) - rows[None, :]            # >0: key above strip start
+        dist_below = rows[None, :] - ((qi[:, None] + 1) * s - 1)  # >0: key below strip end
+        same = ki[None, :] == qi[:, None]
+        above = (ki[None, :] == qi[:, None] - 1) & (dist_above <= r)
+        below = (ki[None, :] == qi[:, None] + 1) & (dist_below <= r)
+        img = same | above | below
+    else:
+        raise ValueError(geometry)
+    if G:
+        img = np.concatenate([img, np.ones((N, G), dtype=bool)], axis=1)
+    return img
+
+
+def dense_attention(q, k, v, *, geometry: str, B, heads, H, W, d, gk=None, gv=None, G=0,
+                    **geom) -> np.ndarray:
+    """Masked-softmax attention over all keys, float64, ``[B, heads, N, d]``."""
+    mask = dense_mask(geometry, H, W, G=G, **geom)
+    Q = bf16_to_f64(q).reshape(B, heads, H * W, d)
+    K = bf16_to_f64(k).reshape(B, heads, H * W, d)
+    V = bf16_to_f64(v).reshape(B, heads, H * W, d)
+    if G:
+        K = np.concatenate([K, bf16_to_f64(gk).reshape(B, heads, G, d)], axis=2)
+        V = np.concatenate([V, bf16_to_f64(gv).reshape(B, heads, G, d)], axis=2)
+    logits = np.einsum("bhtc,bhjc->bhtj", Q, K) / np.sqrt(d)
+    logits = np.where(mask[None, None], logits, -np.inf)
+    logits -= logits.max(axis=-1, keepdims=True)
+    w = np.exp(logits)
+    w /= w.sum(axis=-1, keepdims=True)
+    return np.einsum("bhtj,bhjc->bhtc", w, V)
