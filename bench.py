@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Throughput benchmark of patch-restricted attention on B200.
+
+One step = one forward call of the library (NPA or PCPP, per the workload)
+over the whole synthetic workload, inputs resident in HBM. Prints one JSON
+line (rank 0) with the useful TFLOP/s of all ranks, the roofline of the
+kernel, an end-to-end figure through host buffers, the CPU oracle timed on a
+bounded sample, and the SM clocks seen during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle, as it stands
+
+Multi-GPU (torchrun, one process per GPU): every rank runs the full workload
+as an independent replica (the attention of different images, heads or
+patches needs no exchange), so per-GPU work is fixed and scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import PRESETS, Workload, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "npa_sdxl_4096"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0
+KERNEL_NAME = "npa_fwd_kernel"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(PRESETS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="approximate CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def describe(w: Workload) -> dict:
+    cfg = {"workload": w.name, "B": w.B, "heads": w.heads, "grid": f"{w.H}x{w.W}", "d": w.d}
+    if w.geometry == "npa":
+        cfg.update({"geometry": "npa", "patch": w.patch, "margin": w.margin})
+    else:
+        cfg.update({"geometry": "pcpp", "n_strips": w.n_strips, "p": w.p})
+    cfg["global_tokens"] = w.G
+    if w.smooth_k:
+        cfg["k"] = "3x3 box-filtered"
+    return cfg
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "patch_res_diffusion_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def useful_flops(w: Workload) -> float:
+    import patch_res_diffusion_b200 as npa
+    if w.geometry == "npa":
+        return npa.npa_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
+    return npa.pcpp_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, w.G)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+
+def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
+    """Times the float64 oracle on a growing random query sample until about
+    ``seconds`` of wall time; returns useful TFLOP/s and what was sampled."""
+    import oracle
+    rng = np.random.default_rng(123)
+    N = w.H * w.W
+    geom = dict(patch=w.patch, margin=w.margin) if w.geometry == "npa" else dict(n_strips=w.n_strips, p=w.p)
+    fn = oracle.npa_attention if w.geometry == "npa" else oracle.pcpp_attention
+    key_count = (lambda t: len(oracle.npa_key_set(w.H, w.W, w.patch, w.margin, t))) if w.geometry == "npa" \
+        else (lambda t: len(oracle.pcpp_key_set(w.H, w.W, w.n_strips, w.p, t)))
+    n, total_q, total_pairs, total_t = 64, 0, 0, 0.0
+    while total_t < seconds:
+        qs = np.stack([rng.integers(w.B, size=n), rng.integers(w.heads, size=n), rng.integers(N, size=n)],
+                      axis=1).astype(np.int32)
+        pairs = sum(key_count(int(t)) + w.G for t in qs[:, 2])
+        t0 = time.perf_counter()
+        fn(inp["q"], inp["k"], inp["v"], gk=inp.get("gk"), gv=inp.get("gv"), G=w.G, B=w.B, heads=w.heads,
+           H=w.H, W=w.W, d=w.d, queries=qs, **geom)
+        dt = time.perf_counter() - t0
+        total_q += n
+        total_pairs += pairs
+        total_t += dt
+        n = min(n * 2, 1 << 16)
+    flops = 4.0 * w.d * total_pairs
+    return {
+        "value": flops / total_t / 1e12,
+        "unit": "TFLOP/s",
+        "cores": oracle.num_threads(),
+        "kind": "oracle",
+        "sample": f"{total_q} uniformly drawn (b, h, query) rows of {w.name}, float64, {total_t:.1f} s",
+        "seconds": total_t,
+    }
+
+
+def run_reference(args, w: Workload, rank: int) -> None:
+    if rank != 0:
+        return
+    inp = make_inputs(w)
+    steps = []
+    budget = max(1.0, 30.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        r = oracle_rate(w, inp, budget)
+        if i >= args.warmup:
+            steps.append(r)
+    value = statistics.median(r["value"] for r in steps)
+    flops_step = useful_flops_host(w)
+    line = {
+        "impl": "reference",
+        "metric": "patch-attention useful TFLOP/s (bf16) and % of B200 dense BF16 peak",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": flops_step / (value * 1e12) * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": describe(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": steps[0]["cores"], "kind": "oracle",
+                         "sample": "each step: " + steps[-1]["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "ms_per_step is projected from the sampled rate to the full workload",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def useful_flops_host(w: Workload) -> float:
+    import oracle
+    pairs = oracle.pair_count(w.geometry, w.H, w.W, patch=w.patch, margin=w.margin, n_strips=w.n_strips,
+                              p=w.p, G=w.G)
+    return 4.0 * w.d * w.B * w.heads * pairs
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"npa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
+                                 "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
+                                 "sw_power": parts[8]})
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 300.0] or rows
+        reasons = set()
+        for r in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                              ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(loaded),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# The GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+    import patch_res_diffusion_b200 as npa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = make_inputs(w)
+
+    def dev_bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v = dev_bf16(inp["q"]), dev_bf16(inp["k"]), dev_bf16(inp["v"])
+    gk = dev_bf16(inp["gk"]) if w.G else None
+    gv = dev_bf16(inp["gv"]) if w.G else None
+    o = torch.empty_like(q)
+    stream = torch.cuda.current_stream(dev)
+    flops = useful_flops(w)
+    bytes_io = (q.numel() * 4 + (2 * gk.numel() if w.G else 0)) * 2  # q, k, v, o (+ global k, v)
+    needs_flush = bytes_io < 2 * L2_BYTES
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if needs_flush else None
+
+    def call():
+        if w.geometry == "npa":
+            npa.npa_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, gk, gv, w.G, stream)
+        else:
+            npa.pcpp_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, gk, gv, w.G, stream)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.fill_(1)
+        call()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t_begin.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        starts[i].record(stream)
+        call()
+        ends[i].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    status = npa.npa_device_status(stream)
+    if status != npa.NPA_OK:
+        raise RuntimeError(f"device status {npa.npa_status_string(status)}")
+
+    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernel_ms_sum = sum(kernel_ms)
+    elapsed_ms = t_begin.elapsed_time(t_end)
+    timed_ms = kernel_ms_sum if flush is not None else elapsed_ms
+    if world > 1:
+        t = torch.tensor([timed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        timed_ms = float(t.item())
+    value = world * flops * args.steps / (timed_ms * 1e-3) / 1e12
+    avg_kernel_ms = kernel_ms_sum / args.steps
+
+    # end to end through host buffers: H2D of the inputs, the call, D2H of O
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.to("cpu").pin_memory() for x in (q, k, v))
+        hg = [x.to("cpu").pin_memory() for x in (gk, gv)] if w.G else []
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(x.numel() * 2 for x in [hq, hk, hv] + hg)
+        d2h = ho.numel() * 2
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            if w.G:
+                gk.copy_(hg[0], non_blocking=True)
+                gv.copy_(hg[1], non_blocking=True)
+            call()
+            ho.copy_(o, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * flops * args.steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    achieved = flops / (avg_kernel_ms * 1e-3) / 1e12
+    roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+        "frac": achieved / pk["bf16_tflops"], "traffic": recorded_traffic(w.name),
+        "peak_kind": f"{pk_kind} bf16 burst",
+        "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
+        "frac_of_datasheet_dense": achieved / DATASHEET_BF16_DENSE_TFLOPS,
+        "kernel": KERNEL_NAME, "useful_flops_per_launch": flops,
+        "avg_launch_ms": avg_kernel_ms,
+        "hbm_min_bytes_per_launch": bytes_io,
+    }
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        cpu = oracle_rate(w, inp, args.cpu_seconds)
+        cpu.pop("seconds", None)
+    cfg = describe(w)
+    cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+    cfg["l2"] = ("flushed (256 MB write) between launches; value from per-launch events" if flush is not None
+                 else f"inputs larger than L2 ({bytes_io / 2**20:.0f} MiB touched per launch)")
+    line = {
+        "metric": "patch-attention useful TFLOP/s (bf16) and % of B200 dense BF16 peak",
+        "value": value,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": timed_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": cfg,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk,
+        "gpu_launches": args.steps,
+        "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = PRESETS[args.workload]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

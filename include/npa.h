@@ -1,0 +1,126 @@
+/*
+ * npa.h - C ABI of the B200 (sm_100a) patch-restricted self-attention library.
+ *
+ * The library computes the forward pass of softmax self-attention in which
+ * every query token sees only a restricted, geometry-defined set of keys:
+ *
+ *  - Neighborhood Patch Attention (NPA). ScaleDiff: Higher-Resolution Image
+ *    Synthesis via Efficient and Model-Agnostic Diffusion (atlas.scime.ai
+ *    summary), opening summary and "Approach": the latent token grid is cut
+ *    into non-overlapping square query patches; each patch attends to an
+ *    overlapping key/value neighbourhood. Here the neighbourhood is the patch
+ *    grown by `margin` tokens on every side and clipped to the grid (border
+ *    windows are smaller; they are not shifted inward). When `patch` does not
+ *    divide H or W the last patch row/column is smaller.
+ *
+ *  - Partially conditioned attention (PCPP). Partially Conditioned Patch
+ *    Parallelism for Accelerated Diffusion Model Inference (pith.science
+ *    review), "What carries the argument" and "Core claim": the grid is cut
+ *    into `n_strips` horizontal strips of s = H / n_strips rows; a strip
+ *    attends to its own rows plus the p-fraction of each adjacent strip's
+ *    height that touches it (the bottom rows of the strip above, the top rows
+ *    of the strip below). The row count is r = ceil(p * s) evaluated in double
+ *    with a 1e-9 allowance (so 0.3 * 10 gives 3), limited to s.
+ *
+ *  - Either geometry may append G global tokens (for example joint text
+ *    tokens) to every key/value set. Global tokens produce no output rows.
+ *
+ * Arithmetic: bfloat16 inputs, float32 accumulation of Q.K^T and P.V on the
+ * tensor cores, float32 online softmax with scale 1/sqrt(d), bfloat16 output
+ * rounded to nearest even. Softmax probabilities are rounded to bfloat16
+ * before the P.V product.
+ *
+ * Layouts (all row-major, contiguous, little endian, 16-byte aligned):
+ *   q, k, v, o : bfloat16 [B, heads, H*W, d], token t = row*W + col
+ *   global k, v: bfloat16 [B, heads, G, d]
+ *
+ * Ownership and ordering: the caller owns every buffer. Calls are
+ * asynchronous and ordered on `stream` (NULL = the legacy default stream);
+ * buffers must stay valid until the stream reaches the call. The compute
+ * entry points allocate no device memory; the library's only device state is
+ * one status word per device (see npa_device_status). Host-side state is
+ * limited to per-device capability checks and kernel attributes, set up under
+ * a lock on first use, so the entry points are safe to call from several host
+ * threads.
+ *
+ * Errors: every entry point validates its arguments on the host and returns a
+ * status code; nothing aborts, prints or throws across this boundary. A
+ * failed launch returns NPA_ERR_CUDA. Device-side waits are bounded; if one
+ * runs out, the kernel stops early, leaves the output undefined and records
+ * NPA_ERR_DEVICE_TIMEOUT in the device status word.
+ */
+#ifndef NPA_B200_H
+#define NPA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *npa_stream_t;
+
+typedef enum {
+    NPA_OK = 0,
+    NPA_ERR_INVALID_ARG = 1,     /* null pointer, size < 1, bad p, overlap, H % n_strips != 0 */
+    NPA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, size beyond limits, device not sm_100 */
+    NPA_ERR_MISALIGNED = 3,      /* a pointer is not 16-byte aligned */
+    NPA_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
+    NPA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait ran out */
+} npa_status;
+
+/* Optional global tokens appended to every key/value set.
+ * k, v: bfloat16 [B, heads, n_tokens, d], device memory.
+ * Pass NULL, or n_tokens = 0, for none. */
+typedef struct {
+    const void *k;
+    const void *v;
+    int n_tokens;
+} npa_global_kv;
+
+/* Neighborhood Patch Attention forward (ScaleDiff summary, "Approach").
+ * q, k, v, o: device pointers, layout above; o must not overlap q, k, v or the
+ * global tokens. patch >= 1 (query patch side in tokens), margin >= 0 (window
+ * growth in tokens on each side). d must be 64 or 128. */
+npa_status npa_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                             int B, int heads, int H, int W, int d, int patch, int margin,
+                             const npa_global_kv *global_kv, npa_stream_t stream);
+
+/* Partially conditioned attention forward (PCPP review, "What carries the
+ * argument"). n_strips >= 1 must divide H; 0 <= p <= 1 is the partial value.
+ * Other arguments as for npa_attention_fwd. */
+npa_status pcpp_attention_fwd(const void *q, const void *k, const void *v, void *o,
+                              int B, int heads, int H, int W, int d, int n_strips, double p,
+                              const npa_global_kv *global_kv, npa_stream_t stream);
+
+/* r = ceil(p * strip_rows) (double, 1e-9 allowance), limited to
+ * [0, strip_rows]. Returns -1 if strip_rows < 1 or p is outside [0, 1]. */
+int pcpp_neighbor_rows(int strip_rows, double p);
+
+/* Useful floating-point work of one call: 4 * d * B * heads * (sum over
+ * queries of the key-set size, global keys included) - two multiply-adds per
+ * (query, key, channel) for Q.K^T and P.V; softmax work not counted.
+ * Returns a negative value for invalid geometry arguments. */
+double npa_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G);
+double pcpp_useful_flops(int B, int heads, int H, int W, int d, int n_strips, double p, int G);
+
+/* Waits for `stream`, then reads and clears the current device's status word:
+ * NPA_OK, or the first device-side error recorded since the last read. */
+npa_status npa_device_status(npa_stream_t stream);
+
+/* Diagnostic: launches one block that waits on a barrier nothing ever
+ * arrives at, with a bounded wait of `limit_us` microseconds (1..1000000),
+ * so the bounded-wait path can be exercised without hanging a GPU. The
+ * expected outcome is that npa_device_status() then returns
+ * NPA_ERR_DEVICE_TIMEOUT. Returns NPA_ERR_INVALID_ARG for a bad limit. */
+npa_status npa_selftest_wait_timeout(uint32_t limit_us, npa_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *npa_status_string(npa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NPA_B200_H */

@@ -1,0 +1,193 @@
+"""B200 (sm_100a) patch-restricted self-attention: Python binding.
+
+A thin ctypes layer over the C ABI in ``include/npa.h`` (``libnpa_b200.so``,
+built in-tree by ``patch_res_diffusion_b200.build``). The functions below carry
+the C names and only marshal arguments; every step of the computation runs in
+the library's CUDA kernels. There is no fallback: if the library is missing or
+a call fails, an exception is raised.
+
+* ``npa_attention_fwd`` - Neighborhood Patch Attention (ScaleDiff summary,
+  "Approach"): non-overlapping query patches, each attending to its patch
+  grown by a margin and clipped to the grid.
+* ``pcpp_attention_fwd`` - partially conditioned attention (PCPP review, "What
+  carries the argument"): row strips attending to themselves plus the nearest
+  ceil(p * rows) rows of each adjacent strip.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "NpaError", "lib", "LIB_PATH", "NPA_OK", "NPA_ERR_INVALID_ARG", "NPA_ERR_UNSUPPORTED",
+    "NPA_ERR_MISALIGNED", "NPA_ERR_CUDA", "NPA_ERR_DEVICE_TIMEOUT", "npa_attention_fwd",
+    "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops", "pcpp_useful_flops",
+    "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string", "npa_attention",
+    "pcpp_attention", "EXPORTED_SYMBOLS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
+
+NPA_OK = 0
+NPA_ERR_INVALID_ARG = 1
+NPA_ERR_UNSUPPORTED = 2
+NPA_ERR_MISALIGNED = 3
+NPA_ERR_CUDA = 4
+NPA_ERR_DEVICE_TIMEOUT = 5
+
+EXPORTED_SYMBOLS = (
+    "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops",
+    "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
+)
+
+
+class NpaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {npa_status_string(code)} ({code})")
+        self.code = code
+
+
+class _GlobalKV(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("n_tokens", ctypes.c_int)]
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library. Raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m patch_res_diffusion_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+        gkv = ctypes.POINTER(_GlobalKV)
+        L.npa_attention_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, gkv, vp]
+        L.npa_attention_fwd.restype = i
+        L.pcpp_attention_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, d, gkv, vp]
+        L.pcpp_attention_fwd.restype = i
+        L.pcpp_neighbor_rows.argtypes = [i, d]
+        L.pcpp_neighbor_rows.restype = i
+        L.npa_useful_flops.argtypes = [i, i, i, i, i, i, i, i]
+        L.npa_useful_flops.restype = d
+        L.pcpp_useful_flops.argtypes = [i, i, i, i, i, i, d, i]
+        L.pcpp_useful_flops.restype = d
+        L.npa_device_status.argtypes = [vp]
+        L.npa_device_status.restype = i
+        L.npa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
+        L.npa_selftest_wait_timeout.restype = i
+        L.npa_status_string.argtypes = [i]
+        L.npa_status_string.restype = ctypes.c_char_p
+        _LIB = L
+    return _LIB
+
+
+def _ptr(x) -> Optional[int]:
+    """Device address of a tensor (``data_ptr``) or a raw integer address."""
+    if x is None:
+        return None
+    if hasattr(x, "data_ptr"):
+        return int(x.data_ptr())
+    return int(x)
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return int(torch.cuda.current_stream().cuda_stream)
+        except ImportError:
+            pass
+        return None
+    if hasattr(stream, "cuda_stream"):
+        return int(stream.cuda_stream)
+    return int(stream)
+
+
+def _gkv(global_k, global_v, n_tokens: int):
+    if not n_tokens:
+        return None
+    return ctypes.byref(_GlobalKV(_ptr(global_k), _ptr(global_v), int(n_tokens)))
+
+
+def _check(code: int, what: str) -> None:
+    if code != NPA_OK:
+        raise NpaError(code, what)
+
+
+def npa_attention_fwd(q, k, v, o, B: int, heads: int, H: int, W: int, d: int, patch: int, margin: int,
+                      global_k=None, global_v=None, n_global: int = 0, stream=None) -> None:
+    """C ``npa_attention_fwd``: bf16 [B, heads, H*W, d] device buffers."""
+    _check(lib().npa_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, heads, H, W, d, patch, margin,
+                                   _gkv(global_k, global_v, n_global), _stream(stream)),
+           "npa_attention_fwd")
+
+
+def pcpp_attention_fwd(q, k, v, o, B: int, heads: int, H: int, W: int, d: int, n_strips: int, p: float,
+                       global_k=None, global_v=None, n_global: int = 0, stream=None) -> None:
+    """C ``pcpp_attention_fwd``: bf16 [B, heads, H*W, d] device buffers."""
+    _check(lib().pcpp_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, heads, H, W, d, n_strips,
+                                    float(p), _gkv(global_k, global_v, n_global), _stream(stream)),
+           "pcpp_attention_fwd")
+
+
+def pcpp_neighbor_rows(strip_rows: int, p: float) -> int:
+    return int(lib().pcpp_neighbor_rows(strip_rows, float(p)))
+
+
+def npa_useful_flops(B, heads, H, W, d, patch, margin, G=0) -> float:
+    return float(lib().npa_useful_flops(B, heads, H, W, d, patch, margin, G))
+
+
+def pcpp_useful_flops(B, heads, H, W, d, n_strips, p, G=0) -> float:
+    return float(lib().pcpp_useful_flops(B, heads, H, W, d, n_strips, float(p), G))
+
+
+def npa_device_status(stream=None) -> int:
+    return int(lib().npa_device_status(_stream(stream)))
+
+
+def npa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib().npa_selftest_wait_timeout(int(limit_us), _stream(stream)), "npa_selftest_wait_timeout")
+
+
+def npa_status_string(code: int) -> str:
+    try:
+        return lib().npa_status_string(int(code)).decode()
+    except ImportError:
+        return f"status {code}"
+
+
+# ---------------------------------------------------------------------------
+# torch conveniences (allocation of the output only; the call is the C one)
+# ---------------------------------------------------------------------------
+
+def _shape(q, H, W):
+    if q.dim() != 4 or q.shape[2] != H * W:
+        raise ValueError(f"expected [B, heads, H*W={H * W}, d], got {tuple(q.shape)}")
+    return int(q.shape[0]), int(q.shape[1]), int(q.shape[3])
+
+
+def npa_attention(q, k, v, H: int, W: int, patch: int, margin: int, global_k=None, global_v=None,
+                  out=None, stream=None):
+    """NPA forward on torch bf16 CUDA tensors [B, heads, H*W, d]; returns ``out``."""
+    B, heads, d = _shape(q, H, W)
+    if out is None:
+        out = q.new_empty(q.shape)
+    G = 0 if global_k is None else int(global_k.shape[2])
+    npa_attention_fwd(q, k, v, out, B, heads, H, W, d, patch, margin, global_k, global_v, G, stream)
+    return out
+
+
+def pcpp_attention(q, k, v, H: int, W: int, n_strips: int, p: float, global_k=None, global_v=None,
+                   out=None, stream=None):
+    """PCPP forward on torch bf16 CUDA tensors [B, heads, H*W, d]; returns ``out``."""
+    B, heads, d = _shape(q, H, W)
+    if out is None:
+        out = q.new_empty(q.shape)
+    G = 0 if global_k is None else int(global_k.shape[2])
+    pcpp_attention_fwd(q, k, v, out, B, heads, H, W, d, n_strips, p, global_k, global_v, G, stream)
+    return out

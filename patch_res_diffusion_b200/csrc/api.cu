@@ -1,0 +1,330 @@
+// api.cu - host side of the C ABI declared in include/npa.h: argument
+// validation, geometry resolution, TMA tensor-map encoding and the launch of
+// the sm_100a kernel. Nothing here computes attention.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "npa.h"
+#include "npa_fwd_kernel.cuh"
+
+namespace {
+
+using npa::FwdParams;
+
+// The kernel's bounded waits give up after this long (a healthy wait is far
+// below a millisecond).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+    bool checked = false;
+    npa_status status = NPA_ERR_UNSUPPORTED;
+};
+DeviceState g_dev[kMaxDevices];
+
+// Resolves the tensor-map encoder and checks (once per device) that the
+// current device is an sm_100 part; sets the kernels' shared-memory limits.
+npa_status ensure_ready() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NPA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return NPA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) != cudaSuccess ||
+            qres != cudaDriverEntryPointSuccess || fn == nullptr)
+            return NPA_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    DeviceState &ds = g_dev[dev];
+    if (!ds.checked) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return NPA_ERR_CUDA;
+        if (major != 10 || minor != 0) {
+            ds.status = NPA_ERR_UNSUPPORTED;
+        } else if (cudaFuncSetAttribute(npa::npa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        npa::KCfg<64>::kSmemBytes) != cudaSuccess ||
+                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        npa::KCfg<128>::kSmemBytes) != cudaSuccess) {
+            return NPA_ERR_CUDA;
+        } else {
+            ds.status = NPA_OK;
+        }
+        ds.checked = true;
+    }
+    return ds.status;
+}
+
+// Rectangle form of both geometries (see npa_geometry.cuh).
+struct Geo {
+    int H, W, Ph, Pw, mh, mw;
+};
+
+// Sum over the patches along one axis of (patch extent) x (window extent).
+long long axis_pair_sum(int L, int P, int m) {
+    long long s = 0;
+    for (int p0 = 0; p0 < L; p0 += P) {
+        const int p1 = p0 + P < L ? p0 + P : L;
+        const int w0 = p0 - m > 0 ? p0 - m : 0;
+        const int w1 = p1 + m < L ? p1 + m : L;
+        s += (long long)(p1 - p0) * (w1 - w0);
+    }
+    return s;
+}
+
+// Sum over the patches along one axis of the window extent padded to `tile`.
+long long axis_window_sum(int L, int P, int m, int tile, bool padded) {
+    long long s = 0;
+    for (int p0 = 0; p0 < L; p0 += P) {
+        const int p1 = p0 + P < L ? p0 + P : L;
+        const int w0 = p0 - m > 0 ? p0 - m : 0;
+        const int w1 = p1 + m < L ? p1 + m : L;
+        const int e = w1 - w0;
+        s += padded ? (long long)((e + tile - 1) / tile) * tile : e;
+    }
+    return s;
+}
+
+// Key block shape: 2^lg columns x 128/2^lg rows, chosen to waste the fewest
+// key slots over all windows (ties go to the wider box: longer contiguous runs).
+int choose_kc_log2(const Geo &g) {
+    int best_lg = 7;
+    long long best_waste = LLONG_MAX;
+    const long long exact = axis_window_sum(g.W, g.Pw, g.mw, 1, false) * axis_window_sum(g.H, g.Ph, g.mh, 1, false);
+    for (int lg = 7; lg >= 4; --lg) {
+        const int kc = 1 << lg, kr = 128 >> lg;
+        const long long padded =
+            axis_window_sum(g.W, g.Pw, g.mw, kc, true) * axis_window_sum(g.H, g.Ph, g.mh, kr, true);
+        if (padded - exact < best_waste) {
+            best_waste = padded - exact;
+            best_lg = lg;
+        }
+    }
+    return best_lg;
+}
+
+// Query tile shape: qc patch columns x qr patch rows (qc*qr <= 128), chosen to
+// need the fewest tiles per patch.
+void choose_q_tile(int Ph, int Pw, int *qc_out, int *qr_out) {
+    const int cands[6] = {Pw < 128 ? Pw : 128, 128, 64, 32, 16, 8};
+    long long best = LLONG_MAX;
+    int bc = 128, br = 1;
+    for (int i = 0; i < 6; ++i) {
+        const int c = cands[i];
+        if (c < 1 || c > 128) continue;
+        int r = 128 / c;
+        if (r > Ph) r = Ph;
+        if (r < 1) r = 1;
+        const long long tiles = (long long)((Pw + c - 1) / c) * ((Ph + r - 1) / r);
+        if (tiles < best) {
+            best = tiles;
+            bc = c;
+            br = r;
+        }
+    }
+    *qc_out = bc;
+    *qr_out = br;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+bool encode(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64_t *dims, const cuuint64_t *strides,
+            const cuuint32_t *box) {
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+npa_status validate_common(const void *q, const void *k, const void *v, void *o, int B, int heads, int H, int W,
+                           int d, const npa_global_kv *gkv, int *G_out) {
+    if (!q || !k || !v || !o) return NPA_ERR_INVALID_ARG;
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1) return NPA_ERR_INVALID_ARG;
+    int G = 0;
+    if (gkv && gkv->n_tokens != 0) {
+        if (gkv->n_tokens < 0 || !gkv->k || !gkv->v) return NPA_ERR_INVALID_ARG;
+        G = gkv->n_tokens;
+    }
+    if (d != 64 && d != 128) return NPA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return NPA_ERR_MISALIGNED;
+    if (G && (!aligned16(gkv->k) || !aligned16(gkv->v))) return NPA_ERR_MISALIGNED;
+    const long long N = (long long)H * W;
+    const long long BH = (long long)B * heads;
+    // tensor-map limits (strides < 2^40 bytes) and 32-bit unit/coordinate math
+    if (N * d * 2 >= (1LL << 40) || BH > INT_MAX / 4 || N > INT_MAX || (long long)G * d * 2 >= (1LL << 40))
+        return NPA_ERR_UNSUPPORTED;
+    const size_t bytes = (size_t)(BH * N * d * 2);
+    const size_t gbytes = (size_t)(BH * G * d * 2);
+    if (overlaps(o, bytes, q, bytes) || overlaps(o, bytes, k, bytes) || overlaps(o, bytes, v, bytes))
+        return NPA_ERR_INVALID_ARG;
+    if (G && (overlaps(o, bytes, gkv->k, gbytes) || overlaps(o, bytes, gkv->v, gbytes))) return NPA_ERR_INVALID_ARG;
+    *G_out = G;
+    return NPA_OK;
+}
+
+npa_status launch(const void *q, const void *k, const void *v, void *o, int B, int heads, int d, const Geo &g,
+                  int G, const npa_global_kv *gkv, npa_stream_t stream) {
+    npa_status st = ensure_ready();
+    if (st != NPA_OK) return st;
+
+    FwdParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.o = o;
+    prm.H = g.H;
+    prm.W = g.W;
+    prm.G = G;
+    prm.Ph = g.Ph;
+    prm.Pw = g.Pw;
+    prm.mh = g.mh;
+    prm.mw = g.mw;
+    prm.nPh = (g.H + g.Ph - 1) / g.Ph;
+    prm.nPw = (g.W + g.Pw - 1) / g.Pw;
+    choose_q_tile(g.Ph, g.Pw, &prm.qc, &prm.qr);
+    prm.tiles_c = (g.Pw + prm.qc - 1) / prm.qc;
+    prm.tiles_r = (g.Ph + prm.qr - 1) / prm.qr;
+    prm.kc_log2 = choose_kc_log2(g);
+    prm.kr = 128 >> prm.kc_log2;
+    prm.n_qblocks = (prm.tiles_c * prm.tiles_r + 1) / 2;
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    prm.wait_limit_ns = kWaitLimitNs;
+
+    const long long units = (long long)B * heads * prm.nPh * prm.nPw * prm.n_qblocks;
+    if (units > INT_MAX || (long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
+
+    const int BH = B * heads;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)BH};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)g.W * d * 2, (cuuint64_t)g.H * g.W * d * 2};
+    const cuuint32_t qbox[4] = {64, (cuuint32_t)prm.qc, (cuuint32_t)prm.qr, 1};
+    const cuuint32_t kbox[4] = {64, (cuuint32_t)(1 << prm.kc_log2), (cuuint32_t)prm.kr, 1};
+    if (!encode(&prm.tm_q, q, 4, dims, strides, qbox) || !encode(&prm.tm_k, k, 4, dims, strides, kbox) ||
+        !encode(&prm.tm_v, v, 4, dims, strides, kbox))
+        return NPA_ERR_CUDA;
+    if (G > 0) {
+        const cuuint64_t gdims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)BH};
+        const cuuint64_t gstrides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
+        const cuuint32_t gbox[3] = {64, 128, 1};
+        if (!encode(&prm.tm_gk, gkv->k, 3, gdims, gstrides, gbox) ||
+            !encode(&prm.tm_gv, gkv->v, 3, gdims, gstrides, gbox))
+            return NPA_ERR_CUDA;
+    }
+
+    void *args[1] = {&prm};
+    cudaError_t e;
+    if (d == 64)
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3((unsigned)units), dim3(320), args,
+                             npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
+    else
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3((unsigned)units), dim3(320), args,
+                             npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
+    return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
+}
+
+int neighbor_rows(int s, double p) {
+    if (s < 1 || !(p >= 0.0) || !(p <= 1.0)) return -1;
+    int r = (int)std::ceil(p * (double)s - 1e-9);
+    if (r < 0) r = 0;
+    if (r > s) r = s;
+    return r;
+}
+
+double useful_flops(int B, int heads, int d, const Geo &g, int G) {
+    const double pairs = (double)axis_pair_sum(g.H, g.Ph, g.mh) * (double)axis_pair_sum(g.W, g.Pw, g.mw) +
+                         (double)g.H * g.W * G;
+    return 4.0 * d * (double)B * heads * pairs;
+}
+
+}  // namespace
+
+extern "C" {
+
+npa_status npa_attention_fwd(const void *q, const void *k, const void *v, void *o, int B, int heads, int H, int W,
+                             int d, int patch, int margin, const npa_global_kv *global_kv, npa_stream_t stream) {
+    int G = 0;
+    npa_status st = validate_common(q, k, v, o, B, heads, H, W, d, global_kv, &G);
+    if (st != NPA_OK) return st;
+    if (patch < 1 || margin < 0) return NPA_ERR_INVALID_ARG;
+    const Geo g{H, W, patch, patch, margin, margin};
+    return launch(q, k, v, o, B, heads, d, g, G, global_kv, stream);
+}
+
+npa_status pcpp_attention_fwd(const void *q, const void *k, const void *v, void *o, int B, int heads, int H, int W,
+                              int d, int n_strips, double p, const npa_global_kv *global_kv, npa_stream_t stream) {
+    int G = 0;
+    npa_status st = validate_common(q, k, v, o, B, heads, H, W, d, global_kv, &G);
+    if (st != NPA_OK) return st;
+    if (n_strips < 1 || H % n_strips != 0 || !(p >= 0.0) || !(p <= 1.0)) return NPA_ERR_INVALID_ARG;
+    const int s = H / n_strips;
+    const Geo g{H, W, s, W, neighbor_rows(s, p), 0};
+    return launch(q, k, v, o, B, heads, d, g, G, global_kv, stream);
+}
+
+int pcpp_neighbor_rows(int strip_rows, double p) { return neighbor_rows(strip_rows, p); }
+
+double npa_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || patch < 1 || margin < 0 || G < 0) return -1.0;
+    return useful_flops(B, heads, d, Geo{H, W, patch, patch, margin, margin}, G);
+}
+
+double pcpp_useful_flops(int B, int heads, int H, int W, int d, int n_strips, double p, int G) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || n_strips < 1 || H % n_strips != 0 || G < 0) return -1.0;
+    const int s = H / n_strips;
+    const int r = neighbor_rows(s, p);
+    if (r < 0) return -1.0;
+    return useful_flops(B, heads, d, Geo{H, W, s, W, r, 0}, G);
+}
+
+npa_status npa_device_status(npa_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return NPA_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, npa::g_npa_status, sizeof(v)) != cudaSuccess) return NPA_ERR_CUDA;
+    if (v != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(npa::g_npa_status, &zero, sizeof(zero)) != cudaSuccess) return NPA_ERR_CUDA;
+    }
+    return (npa_status)v;
+}
+
+npa_status npa_selftest_wait_timeout(uint32_t limit_us, npa_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return NPA_ERR_INVALID_ARG;
+    npa_status st = ensure_ready();
+    if (st != NPA_OK) return st;
+    unsigned long long ns = (unsigned long long)limit_us * 1000ull;
+    void *args[1] = {&ns};
+    cudaError_t e = cudaLaunchKernel((const void *)npa::npa_wait_selftest_kernel, dim3(1), dim3(32), args, 0,
+                                     (cudaStream_t)stream);
+    return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
+}
+
+const char *npa_status_string(npa_status status) {
+    switch (status) {
+        case NPA_OK: return "NPA_OK";
+        case NPA_ERR_INVALID_ARG: return "NPA_ERR_INVALID_ARG";
+        case NPA_ERR_UNSUPPORTED: return "NPA_ERR_UNSUPPORTED";
+        case NPA_ERR_MISALIGNED: return "NPA_ERR_MISALIGNED";
+        case NPA_ERR_CUDA: return "NPA_ERR_CUDA";
+        case NPA_ERR_DEVICE_TIMEOUT: return "NPA_ERR_DEVICE_TIMEOUT";
+    }
+    return "NPA_ERR_UNKNOWN";
+}
+
+}  // extern "C"

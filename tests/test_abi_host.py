@@ -1,0 +1,144 @@
+"""The C-ABI library on the host: it loads, exports every symbol the header
+declares, validates arguments before touching a GPU, and its geometry helpers
+agree with the oracle's brute-force counts. No compute call is made here."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+import patch_res_diffusion_b200 as npa
+from workloads import PRESETS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "npa.h")
+
+
+def header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(",
+                                 src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from patch_res_diffusion_b200 import build
+    build.build()
+    return npa.lib()
+
+
+def test_header_declares_the_bound_symbols():
+    assert header_functions() == sorted(npa.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_header_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", npa.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(L, name) is not None
+
+
+def test_status_strings(L):
+    for code, name in [(0, "NPA_OK"), (1, "NPA_ERR_INVALID_ARG"), (2, "NPA_ERR_UNSUPPORTED"),
+                       (3, "NPA_ERR_MISALIGNED"), (4, "NPA_ERR_CUDA"), (5, "NPA_ERR_DEVICE_TIMEOUT")]:
+        assert npa.npa_status_string(code) == name
+    assert npa.npa_status_string(99) == "NPA_ERR_UNKNOWN"
+
+
+# fake, never dereferenced addresses: validation rejects these calls before any CUDA call
+A, B_, C_, O_ = 0x10000, 0x20000000, 0x40000000, 0x60000000
+
+
+def _npa(L, q=A, k=B_, v=C_, o=O_, B=1, h=1, H=8, W=8, d=64, P=4, m=1, g=None):
+    return L.npa_attention_fwd(q, k, v, o, B, h, H, W, d, P, m, g, None)
+
+
+def _pcpp(L, q=A, k=B_, v=C_, o=O_, B=1, h=1, H=8, W=8, d=64, n=2, p=0.5, g=None):
+    return L.pcpp_attention_fwd(q, k, v, o, B, h, H, W, d, n, p, g, None)
+
+
+def test_null_and_size_arguments_rejected(L):
+    assert _npa(L, q=None) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, o=None) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, B=0) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, H=0) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, P=0) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, m=-1) == npa.NPA_ERR_INVALID_ARG
+    assert _pcpp(L, n=0) == npa.NPA_ERR_INVALID_ARG
+
+
+def test_unsupported_head_dim(L):
+    for d in (16, 32, 96, 256):
+        assert _npa(L, d=d) == npa.NPA_ERR_UNSUPPORTED
+        assert _pcpp(L, d=d) == npa.NPA_ERR_UNSUPPORTED
+
+
+def test_misaligned_pointers(L):
+    assert _npa(L, q=A + 8) == npa.NPA_ERR_MISALIGNED
+    assert _npa(L, o=O_ + 2) == npa.NPA_ERR_MISALIGNED
+    g = ctypes.byref(npa._GlobalKV(0x70000008, 0x78000000, 5))
+    assert _npa(L, g=g) == npa.NPA_ERR_MISALIGNED
+
+
+def test_overlapping_output_rejected(L):
+    assert _npa(L, o=A + 64) == npa.NPA_ERR_INVALID_ARG
+    assert _pcpp(L, o=C_) == npa.NPA_ERR_INVALID_ARG
+    g = ctypes.byref(npa._GlobalKV(O_ + 16, 0x78000000, 5))
+    assert _npa(L, g=g) == npa.NPA_ERR_INVALID_ARG
+
+
+def test_global_token_arguments(L):
+    assert _npa(L, g=ctypes.byref(npa._GlobalKV(None, 0x78000000, 5))) == npa.NPA_ERR_INVALID_ARG
+    assert _npa(L, g=ctypes.byref(npa._GlobalKV(0x70000000, 0x78000000, -1))) == npa.NPA_ERR_INVALID_ARG
+
+
+def test_pcpp_argument_domain(L):
+    assert _pcpp(L, H=9, n=2) == npa.NPA_ERR_INVALID_ARG          # strips must divide H
+    assert _pcpp(L, p=1.5) == npa.NPA_ERR_INVALID_ARG
+    assert _pcpp(L, p=-0.1) == npa.NPA_ERR_INVALID_ARG
+    assert _pcpp(L, p=float("nan")) == npa.NPA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("s", list(range(1, 70)))
+def test_neighbor_rows_agree_with_oracle(s):
+    for p in np.round(np.linspace(0, 1, 41), 6).tolist() + [0.3, 0.7, 0.8, 1 / 3, 2 / 3]:
+        assert npa.pcpp_neighbor_rows(s, p) == oracle.pcpp_neighbor_rows(s, p), (s, p)
+    assert npa.pcpp_neighbor_rows(s, 1.01) == -1
+
+
+@pytest.mark.parametrize("name", list(PRESETS))
+def test_useful_flops_match_oracle_pair_count(name):
+    w = PRESETS[name]
+    pairs = oracle.pair_count(w.geometry, w.H, w.W, patch=w.patch, margin=w.margin, n_strips=w.n_strips,
+                              p=w.p, G=w.G)
+    expect = 4.0 * w.d * w.B * w.heads * pairs
+    if w.geometry == "npa":
+        got = npa.npa_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
+    else:
+        got = npa.pcpp_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, w.G)
+    assert got == expect
+
+
+@pytest.mark.parametrize("H,W,P,m,G", [(17, 23, 5, 3, 0), (9, 31, 8, 0, 7), (40, 13, 64, 2, 1), (30, 30, 7, 30, 0)])
+def test_useful_flops_ragged_npa(H, W, P, m, G):
+    pairs = oracle.pair_count("npa", H, W, patch=P, margin=m, G=G)
+    assert npa.npa_useful_flops(2, 3, H, W, 128, P, m, G) == 4.0 * 128 * 6 * pairs
+
+
+@pytest.mark.parametrize("H,W,n,p,G", [(30, 7, 5, 0.45, 0), (24, 9, 8, 1.0, 3), (12, 5, 1, 0.5, 0)])
+def test_useful_flops_pcpp(H, W, n, p, G):
+    pairs = oracle.pair_count("pcpp", H, W, n_strips=n, p=p, G=G)
+    assert npa.pcpp_useful_flops(1, 2, H, W, 64, n, p, G) == 4.0 * 64 * 2 * pairs
+
+
+def test_flops_helper_rejects_bad_geometry():
+    assert npa.npa_useful_flops(1, 1, 8, 8, 64, 0, 1) < 0
+    assert npa.pcpp_useful_flops(1, 1, 9, 8, 64, 2, 0.5) < 0
+    assert npa.pcpp_useful_flops(1, 1, 8, 8, 64, 2, 1.5) < 0

@@ -1,0 +1,183 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the
+float64 CPU oracle on the same seeded inputs.
+
+* element by element on small and ragged problems that span several query
+  tiles, several key blocks, partial blocks and a ragged global-token tail;
+* on the full workloads, at the launch configuration the benchmark times,
+  on a deterministic sample of queries the oracle computes one by one;
+* window membership exactly, through probe inputs (q = 0 makes attention
+  uniform over the key set; one-hot values reveal which keys are in it);
+* bitwise determinism, stream ordering, and the bounded-wait status path.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from workloads import PRESETS, Workload, make_inputs, f64_to_bf16_bits
+from _parity import compare, passes, run_gpu, run_oracle, sample_queries, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from patch_res_diffusion_b200 import build
+    build.build()
+    import patch_res_diffusion_b200 as npa
+    npa.lib()
+    yield
+    assert npa.npa_device_status() == npa.NPA_OK
+
+
+SMALL = [
+    Workload("tiny_npa", "npa", B=1, heads=2, H=16, W=16, d=64, patch=8, margin=4),
+    Workload("npa64_p32", "npa", B=1, heads=2, H=64, W=64, d=64, patch=32, margin=16),
+    Workload("npa_ragged", "npa", B=2, heads=1, H=72, W=80, d=64, patch=32, margin=16),
+    Workload("npa_odd_patch", "npa", B=1, heads=2, H=50, W=70, d=64, patch=24, margin=5),
+    Workload("npa_wide_patch", "npa", B=1, heads=1, H=40, W=300, d=64, patch=150, margin=7),
+    Workload("npa_d128_global", "npa", B=1, heads=2, H=64, W=64, d=128, patch=32, margin=16, G=100),
+    Workload("npa_d64_global", "npa", B=1, heads=2, H=48, W=40, d=64, patch=16, margin=8, G=260),
+    Workload("npa_m0", "npa", B=1, heads=2, H=32, W=48, d=64, patch=16, margin=0),
+    Workload("npa_full_window", "npa", B=1, heads=1, H=24, W=20, d=64, patch=8, margin=24),
+    Workload("pcpp_4x16", "pcpp", B=1, heads=2, H=64, W=64, d=64, n_strips=4, p=0.3),
+    Workload("pcpp_8x8", "pcpp", B=1, heads=2, H=64, W=64, d=64, n_strips=8, p=0.8),
+    Workload("pcpp_w96", "pcpp", B=1, heads=2, H=48, W=96, d=64, n_strips=3, p=0.5),
+    Workload("pcpp_w200", "pcpp", B=1, heads=1, H=32, W=200, d=64, n_strips=4, p=0.25),
+    Workload("pcpp_d128_global", "pcpp", B=1, heads=2, H=64, W=64, d=128, n_strips=4, p=0.3, G=77),
+    Workload("pcpp_p0", "pcpp", B=1, heads=1, H=32, W=64, d=64, n_strips=4, p=0.0),
+    Workload("pcpp_p1_two", "pcpp", B=1, heads=1, H=32, W=64, d=64, n_strips=2, p=1.0),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_full_parity(w):
+    inp = make_inputs(w)
+    got = to_f64(run_gpu(w, inp))
+    ref = run_oracle(w, inp)
+    m = compare(got, ref)
+    assert passes(m), m
+
+
+@pytest.mark.parametrize("name", list(PRESETS))
+def test_full_workload_sampled_parity(name):
+    w = PRESETS[name]
+    inp = make_inputs(w)
+    o = run_gpu(w, inp)
+    torch.cuda.synchronize()
+    qs = sample_queries(w, n_random=512, seed=1, max_bh=4 if w.d == 128 else None)
+    ref = run_oracle(w, inp, queries=qs)
+    flat = o.view(w.B * w.heads * w.H * w.W, w.d)
+    idx = torch.from_numpy(((qs[:, 0].astype(np.int64) * w.heads + qs[:, 1]) * (w.H * w.W) + qs[:, 2])).cuda()
+    got = to_f64(flat.index_select(0, idx))
+    m = compare(got, ref)
+    assert passes(m), m
+    # every output row was written (the buffer starts as NaN)
+    assert bool(torch.isfinite(o).all())
+
+
+def _probe_case(w: Workload, probe_keys):
+    """q = 0, k random, v one-hot: channel c carries key probe_keys[c]."""
+    N = w.H * w.W
+    rng = np.random.default_rng(3)
+    q = np.zeros((1, 1, N, w.d), dtype=np.uint16)
+    k = f64_to_bf16_bits(rng.standard_normal((1, 1, N, w.d)))
+    v = np.zeros((1, 1, N, w.d))
+    for c, j in enumerate(probe_keys):
+        v[0, 0, j, c] = 1.0
+    return {"q": q, "k": k, "v": f64_to_bf16_bits(v)}
+
+
+def _probe_keys(w: Workload):
+    N = w.H * w.W
+    rows = sorted({0, 1, w.H - 1, w.H // 2, w.H // 2 - 1, w.H // 3})
+    cols = sorted({0, w.W - 1, w.W // 2, w.W // 3, 7 % w.W})
+    keys = [r * w.W + c for r in rows for c in cols]
+    rng = np.random.default_rng(9)
+    while len(keys) < w.d:
+        keys.append(int(rng.integers(N)))
+    return keys[: w.d]
+
+
+def _key_sets(w: Workload, margin=None, p=None):
+    N = w.H * w.W
+    if w.geometry == "npa":
+        return [set(oracle.npa_key_set(w.H, w.W, w.patch, w.margin if margin is None else margin, t).tolist())
+                for t in range(N)]
+    return [set(oracle.pcpp_key_set(w.H, w.W, w.n_strips, w.p if p is None else p, t).tolist()) for t in range(N)]
+
+
+PROBES = [
+    Workload("probe_npa", "npa", B=1, heads=1, H=40, W=36, d=64, patch=16, margin=5),
+    Workload("probe_npa_tiny", "npa", B=1, heads=1, H=16, W=16, d=64, patch=8, margin=4),
+    Workload("probe_pcpp", "pcpp", B=1, heads=1, H=48, W=40, d=64, n_strips=3, p=0.4),
+    Workload("probe_pcpp_8", "pcpp", B=1, heads=1, H=64, W=32, d=64, n_strips=8, p=0.8),
+]
+
+
+def _membership(w, out, keys):
+    o = to_f64(out)[0, 0]
+    return o, [[o[t, c] > 0 for c in range(len(keys))] for t in range(w.H * w.W)]
+
+
+@pytest.mark.parametrize("w", PROBES, ids=lambda w: w.name)
+def test_probe_window_membership_exact(w):
+    keys = _probe_keys(w)
+    inp = _probe_case(w, keys)
+    out = run_gpu(w, inp)
+    o, member = _membership(w, out, keys)
+    sets = _key_sets(w)
+    for t in range(w.H * w.W):
+        for c, j in enumerate(keys):
+            assert member[t][c] == (j in sets[t]), (t, j)
+            if j in sets[t]:
+                assert abs(o[t, c] * len(sets[t]) - 1.0) < 1e-2
+
+
+def test_probe_negative_control_margin_off_by_one():
+    """The membership probe must tell margin m from m+1."""
+    w = PROBES[0]
+    keys = _probe_keys(w)
+    inp = _probe_case(w, keys)
+    out = run_gpu(w, inp, margin=w.margin + 1)
+    _, member = _membership(w, out, keys)
+    sets = _key_sets(w)
+    mismatches = sum(member[t][c] != (j in sets[t]) for t in range(w.H * w.W) for c, j in enumerate(keys))
+    assert mismatches > 0
+
+
+def test_negative_control_zero_output_fails_gate():
+    w = SMALL[1]
+    ref = run_oracle(w, make_inputs(w))
+    assert not passes(compare(np.zeros_like(ref), ref))
+
+
+def test_bitwise_deterministic():
+    w = SMALL[5]
+    inp = make_inputs(w)
+    a = run_gpu(w, inp)
+    b = run_gpu(w, inp)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_side_stream_ordering():
+    w = SMALL[2]
+    inp = make_inputs(w)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o = run_gpu(w, inp, stream=s)
+    s.synchronize()
+    m = compare(to_f64(o), run_oracle(w, inp))
+    assert passes(m), m
+
+
+def test_bounded_wait_reports_timeout():
+    import patch_res_diffusion_b200 as npa
+    assert npa.npa_device_status() == npa.NPA_OK
+    npa.npa_selftest_wait_timeout(2000)
+    assert npa.npa_device_status() == npa.NPA_ERR_DEVICE_TIMEOUT
+    assert npa.npa_device_status() == npa.NPA_OK  # read clears it
