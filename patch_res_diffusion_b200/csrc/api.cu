@@ -231,10 +231,10 @@ npa_status launch(const void *q, const void *k, const void *v, void *o, int B, i
     void *args[1] = {&prm};
     cudaError_t e;
     if (d == 64)
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3((unsigned)units), dim3(320), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3((unsigned)units), dim3(npa::KCfg<64>::kThreads), args,
                              npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
     else
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3((unsigned)units), dim3(320), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3((unsigned)units), dim3(npa::KCfg<128>::kThreads), args,
                              npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
     return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
 }

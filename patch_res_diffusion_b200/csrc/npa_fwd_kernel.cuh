@@ -2,29 +2,47 @@
 // self-attention (NPA and PCPP share it through npa_geometry.cuh).
 //
 // One CTA per work unit: two 128-query tiles of one patch that share the
-// patch's key/value window. Ten warps, each with one role:
-//   warps 0-3  softmax + epilogue for query tile 0 (TMEM lanes 0..127)
-//   warps 4-7  softmax + epilogue for query tile 1
-//   warp  8    TMA producer (Q once, then K and V blocks through a ring of
-//              kStages shared-memory stages); owns the TMEM allocation
-//   warp  9    MMA issuer (one thread issues every tcgen05.mma)
+// patch's key/value window. Three warpgroups (12 warps):
+//   warps 0-3   softmax + epilogue for query tile 0 (TMEM lanes 0..127)
+//   warps 4-7   softmax + epilogue for query tile 1
+//   warp  8     TMA producer (Q once, then K and V blocks through a ring of
+//               kStages shared-memory stages); owns the TMEM allocation
+//   warp  9     MMA issuer: d = 64, the S = Q K^T products; d = 128, all
+//   warp  10    d = 64: MMA issuer of the O += P V products
+//   warps 10-11 otherwise idle
+// The kernel is launched with 168 registers per thread; the third warpgroup
+// gives registers back (setmaxnreg.dec to kRegsCtl) and the softmax
+// warpgroups take them (setmaxnreg.inc to kRegsSoftmax):
+// 2 * 128 * kRegsSoftmax + 128 * kRegsCtl = 384 * 168, the launch's total.
 //
 // Per key block j and tile q the MMA warp issues S_q = Q_q K_j^T into TMEM
 // (M=128, N=128, K=d, both operands K-major in 128-byte-swizzled shared
 // memory); the softmax warps read S_q from TMEM (one thread per query row),
-// update the running maximum and sum, and write P_q = exp2(S*log2e/sqrt(d) -
-// m) as bf16 back into the first 64 columns of the same TMEM region; the MMA
+// update the running maximum and sum, and write P_q as bf16 into TMEM; the MMA
 // warp then issues O_q += P_q V_j with A = P_q read from TMEM and B = V_j
-// (MN-major, 128-byte swizzle). The issue order PV_q(j-1) -> S_q(j) lets the
-// two tiles ping-pong: the tensor core works on one tile while the softmax
-// warps of the other run. Because tcgen05 operations of one thread complete
-// in order, the commit that announces S_q(j) also guarantees that PV_q(j-1)
-// has finished, so the softmax warps may rescale O_q and overwrite P_q as
-// soon as S_q(j) is visible.
+// (MN-major, 128-byte swizzle).
 //
-// The running maximum is rescaled lazily: O and the row sum are rescaled only
-// when the block maximum exceeds the reference maximum by more than 8 (log2
-// units), which keeps P <= 256 and leaves the final O / l exact.
+// TMEM (512 columns x 128 lanes). d = 64: S0 S1 | O0 O1 | P0 P1, so P has its
+// own buffer and the MMA warp issues S_q(j+1) as soon as the softmax warps
+// have copied S_q(j) into registers: the softmax runs back to back while the
+// tensor core computes the next scores. d = 128: S0 S1 | O0 O1 with P_q in the
+// first 64 columns of S_q; the MMA warp then issues PV_q(j-1) before S_q(j),
+// and because tcgen05 operations of one thread complete in order, the commit
+// that announces S_q(j) also guarantees that PV_q(j-1) has finished. The two
+// tiles ping-pong: the tensor core works on one while the other's softmax runs.
+//
+// Softmax arithmetic per block. The two softmax warpgroups take turns on the
+// exponential unit (MUFU): warpgroup q loads its scores and takes the block
+// maximum (a tree of three-input maxima) while the other group evaluates its
+// exponentials, then waits for its turn, evaluates the block's 128 x 128
+// exponentials and hands the turn back, so one group's loads, stores and
+// barrier traffic overlap the other's exponentials. p = 2^(s*log2(e)/sqrt(d)
+// - R) on the packed f32x2 FMA path and ex2.approx.f32, rounded to bf16 pairs
+// for P and summed in float32 (four packed partial sums). The reference R is
+// moved lazily: only when the block maximum exceeds it by more than
+// kRescaleLog2 (log2 units), in which case O and the row sum are rescaled by
+// 2^(R_old - R_new) before this block's P.V. P <= 2^kRescaleLog2 and the final
+// O / l is exact up to rounding.
 //
 // Every wait is bounded (FwdParams::wait_limit_ns). On expiry the CTA records
 // NPA_ERR_DEVICE_TIMEOUT in the device status word, stops issuing work,
@@ -44,6 +62,7 @@ __device__ unsigned int g_npa_status;  // first device-side error since last rea
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_npa_status, 0u, code); }
 
 constexpr unsigned int kErrDeviceTimeout = 5u;  // NPA_ERR_DEVICE_TIMEOUT
+constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
 template <int D>
 struct KCfg {
@@ -52,7 +71,11 @@ struct KCfg {
     static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
     static constexpr int kTileBytes = kChunks * kChunkBytes;
     static constexpr int kStages = (D == 64) ? 4 : 2;
-    static constexpr int kThreads = 320;
+    static constexpr int kThreads = 384;
+    static constexpr uint32_t kRegsLaunch = 168;
+    static constexpr uint32_t kRegsSoftmax = 216;
+    static constexpr uint32_t kRegsCtl = 72;
+    static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl == kThreads * kRegsLaunch, "register split");
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = 2 * kTileBytes;
     static constexpr int kOffV = kOffK + kStages * kTileBytes;
@@ -63,17 +86,21 @@ struct KCfg {
     static constexpr int bKEmpty = bKFull + kStages;
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
-    static constexpr int bSFull = bVEmpty + kStages;   // [2]
-    static constexpr int bPFull = bSFull + 2;          // [2]
-    static constexpr int bOFinal = bPFull + 2;         // [2]
-    static constexpr int bDrain = bOFinal + 2;
-    static constexpr int kNumBars = bDrain + 1;
+    static constexpr int bSFull = bVEmpty + kStages;   // [2] S_q written (MMA commit)
+    static constexpr int bSFree = bSFull + 2;          // [2] S_q copied to registers (128 arrivals)
+    static constexpr int bPFull = bSFree + 2;          // [2] P_q written (128 arrivals)
+    static constexpr int bPFree = bPFull + 2;          // [2] PV_q done (MMA commit)
+    static constexpr int bTurn = bPFree + 2;           // [2] exponential-phase turn of warpgroup q (4 arrivals)
+    static constexpr int bDrain = bTurn + 2;           // [2] one per MMA-issuing warp
+    static constexpr int kNumBars = bDrain + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
     // tensor memory columns
     static constexpr uint32_t kTmemCols = 512;
+    static constexpr bool kSeparateP = (D == 64);
     __device__ static constexpr uint32_t col_s(int q) { return q ? 128u : 0u; }
     __device__ static constexpr uint32_t col_o(int q) { return 256u + (q ? uint32_t(D) : 0u); }
+    __device__ static constexpr uint32_t col_p(int q) { return kSeparateP ? (384u + (q ? 64u : 0u)) : col_s(q); }
 };
 
 // ---------------------------------------------------------------------------
@@ -155,19 +182,121 @@ __device__ void run_producer(const FwdParams &p, const Work &w, uint8_t *smem, u
 // ---------------------------------------------------------------------------
 // MMA issuer: one thread of warp 9.
 // ---------------------------------------------------------------------------
+// Shared-memory descriptors are built once per operand buffer; stepping
+// through K (16 elements = 32 bytes inside a 128-byte swizzle atom, or the
+// next 64-column block) or through the keys of V only adds a constant to the
+// start-address field.
+template <int D>
+__device__ __forceinline__ void issue_s(uint32_t tmem, int q, uint64_t qdesc, uint64_t kdesc) {
+    using C = KCfg<D>;
+    constexpr uint32_t kIdS = sm100::idesc_bf16_f32(128, 128, false, false);  // S = Q K^T
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = uint64_t(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
+        sm100::mma_ss(tmem + C::col_s(q), qdesc + off, kdesc + off, kIdS, kk > 0 ? 1u : 0u);
+    }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t tmem, int q, uint64_t vdesc, bool accumulate) {
+    using C = KCfg<D>;
+    constexpr uint32_t kIdO = sm100::idesc_bf16_f32(128, D, false, true);  // O += P V, V MN-major
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p(q) + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), kIdO,
+                      (accumulate || kk > 0) ? 1u : 0u);
+}
+
+struct OperandDescs {
+    uint64_t q0, q1, k0, v0;  // Q tiles, K and V stage 0
+    uint64_t stage;           // descriptor increment from one stage to the next
+};
+
+template <int D>
+__device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
+    using C = KCfg<D>;
+    OperandDescs d;
+    // K-major operands: SBO = 8 rows x 128 bytes. V (MN-major): LBO = next
+    // 64-column block, SBO = next 8 keys.
+    d.q0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffQ), 16, 1024);
+    d.q1 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffQ + C::kTileBytes), 16, 1024);
+    d.k0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffK), 16, 1024);
+    d.v0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffV), C::kChunkBytes, 1024);
+    d.stage = uint64_t(C::kTileBytes >> 4);
+    return d;
+}
+
+// d = 64 (P has its own TMEM buffer): the S products and the P.V products
+// touch disjoint tensor memory and shared memory, so two warps issue them
+// independently. This one issues S_0(j), S_1(j) as soon as the softmax warps
+// hold S(j-1) in registers.
+template <int D>
+__device__ void run_mma_s(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+                          volatile uint32_t *abort_flag) {
+    using C = KCfg<D>;
+    const uint64_t lim = p.wait_limit_ns;
+    const OperandDescs dd = make_descs<D>(smem);
+    bool ok = sm100::mbar_wait(&bars[C::bQFull], 0, lim);
+    for (int j = 0; ok && j < w.n_blocks; ++j) {
+        if (*abort_flag) break;
+        const int s = j % C::kStages;
+        ok = sm100::mbar_wait(&bars[C::bKFull + s], (j / C::kStages) & 1, lim);
+        for (int q = 0; ok && q < 2; ++q) {
+            if (j > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (j - 1) & 1, lim);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + s * dd.stage);
+            sm100::tc_commit(&bars[C::bSFull + q]);
+        }
+        if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
+    }
+    if (!ok) {
+        record_error(kErrDeviceTimeout);
+        *abort_flag = 1;
+    }
+    sm100::tc_commit(&bars[C::bDrain]);
+    sm100::mbar_wait(&bars[C::bDrain], 0, lim);
+}
+
+// d = 64: the P.V products, O_q(j) += P_q(j) V(j) as each P_q(j) arrives.
+template <int D>
+__device__ void run_mma_pv(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+                           volatile uint32_t *abort_flag) {
+    using C = KCfg<D>;
+    const uint64_t lim = p.wait_limit_ns;
+    const OperandDescs dd = make_descs<D>(smem);
+    bool ok = true;
+    for (int j = 0; ok && j < w.n_blocks; ++j) {
+        if (*abort_flag) break;
+        const int s = j % C::kStages;
+        ok = sm100::mbar_wait(&bars[C::bVFull + s], (j / C::kStages) & 1, lim);
+        for (int q = 0; ok && q < 2; ++q) {
+            ok = sm100::mbar_wait(&bars[C::bPFull + q], j & 1, lim);
+            if (!ok) break;
+            sm100::tc_fence_after();
+            issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > 0);
+            sm100::tc_commit(&bars[C::bPFree + q]);
+        }
+        if (ok) sm100::tc_commit(&bars[C::bVEmpty + s]);
+    }
+    if (!ok) {
+        record_error(kErrDeviceTimeout);
+        *abort_flag = 1;
+    }
+    sm100::tc_commit(&bars[C::bDrain + 1]);
+    sm100::mbar_wait(&bars[C::bDrain + 1], 0, lim);
+}
+
+// d = 128 (P aliases S): one warp issues everything, PV_q(j-1) before S_q(j)
+// for each tile, so that the completion of S_q(j) also implies PV_q(j-1).
 template <int D>
 __device__ void run_mma(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                         volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
-    constexpr uint32_t kIdS = sm100::idesc_bf16_f32(128, 128, false, false);  // S = Q K^T
-    constexpr uint32_t kIdO = sm100::idesc_bf16_f32(128, D, false, true);     // O += P V, V MN-major
     const uint64_t lim = p.wait_limit_ns;
-    const uint32_t sQ = sm100::smem_u32(smem + C::kOffQ);
-    const uint32_t sK = sm100::smem_u32(smem + C::kOffK);
-    const uint32_t sV = sm100::smem_u32(smem + C::kOffV);
+    const OperandDescs dd = make_descs<D>(smem);
     const int n = w.n_blocks;
     bool ok = sm100::mbar_wait(&bars[C::bQFull], 0, lim);
-    sm100::tc_fence_after();
     for (int j = 0; ok && j <= n; ++j) {
         if (*abort_flag) break;
         if (j < n) {
@@ -179,33 +308,16 @@ __device__ void run_mma(const FwdParams &p, const Work &w, uint8_t *smem, uint64
             if (!ok) break;
         }
         sm100::tc_fence_after();
-#pragma unroll
         for (int q = 0; q < 2; ++q) {
             if (j > 0) {
                 ok = sm100::mbar_wait(&bars[C::bPFull + q], (j - 1) & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                const uint32_t vbase = sV + ((j - 1) % C::kStages) * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    // V block: 16 keys x D, MN-major; LBO = next 64-column block,
-                    // SBO = next group of 8 keys.
-                    const uint64_t bdesc = sm100::sdesc_sw128(vbase + kk * 2048, C::kChunkBytes, 1024);
-                    sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_s(q) + kk * 8, bdesc, kIdO,
-                                  (j > 1 || kk > 0) ? 1u : 0u);
-                }
-                if (j == n) sm100::tc_commit(&bars[C::bOFinal + q]);
+                issue_pv<D>(tmem, q, dd.v0 + ((j - 1) % C::kStages) * dd.stage, j > 1);
+                sm100::tc_commit(&bars[C::bPFree + q]);
             }
             if (j < n) {
-                const uint32_t kbase = sK + (j % C::kStages) * C::kTileBytes;
-                const uint32_t qbase = sQ + q * C::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-                    const uint64_t adesc = sm100::sdesc_sw128(qbase + off, 16, 1024);
-                    const uint64_t bdesc = sm100::sdesc_sw128(kbase + off, 16, 1024);
-                    sm100::mma_ss(tmem + C::col_s(q), adesc, bdesc, kIdS, kk > 0 ? 1u : 0u);
-                }
+                issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + (j % C::kStages) * dd.stage);
                 sm100::tc_commit(&bars[C::bSFull + q]);
             }
         }
@@ -217,7 +329,6 @@ __device__ void run_mma(const FwdParams &p, const Work &w, uint8_t *smem, uint64
         record_error(kErrDeviceTimeout);
         *abort_flag = 1;
     }
-    // Drain: no MMA may still be running when the tensor memory is freed.
     sm100::tc_commit(&bars[C::bDrain]);
     sm100::mbar_wait(&bars[C::bDrain], 0, lim);
 }
@@ -230,51 +341,90 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64
     return __all_sync(0xffffffffu, got);
 }
 
+// Row maximum of 128 scores: eight independent chains of three-input maxima.
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+    float mk[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        float m = sm100::max3(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+        for (int t = 3; t < 15; t += 2) m = sm100::max3(m, s[k + 8 * t], s[k + 8 * t + 8]);
+        mk[k] = fmaxf(m, s[k + 120]);
+    }
+    return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
+}
+
+// p = 2^(s*c - ref) for 128 scores: packed bf16 pairs into pk, float32 sum returned.
+__device__ __forceinline__ float exp_block(const float (&s)[128], float c, float ref, uint32_t (&pk)[64]) {
+    const float neg = (ref == -INFINITY) ? 0.f : -ref;
+    const uint64_t c2 = sm100::pack_f32x2(c, c);
+    const uint64_t m2 = sm100::pack_f32x2(neg, neg);
+    uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
+        float x0, x1;
+        sm100::unpack_f32x2(x2, x0, x1);
+        const float p0 = sm100::ex2_approx(x0), p1 = sm100::ex2_approx(x1);
+        pk[i] = sm100::pack_bf16x2(p0, p1);
+        acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
+    }
+    float a0, a1, b0, b1, c0, c1, d0, d1;
+    sm100::unpack_f32x2(acc[0], a0, a1);
+    sm100::unpack_f32x2(acc[1], b0, b1);
+    sm100::unpack_f32x2(acc[2], c0, c1);
+    sm100::unpack_f32x2(acc[3], d0, d1);
+    return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+}
+
 template <int D>
 __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, uint32_t tmem,
                             volatile uint32_t *abort_flag, int q) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     const int row = threadIdx.x & 127;
+    const bool lane0 = (threadIdx.x & 31) == 0;
     const uint32_t lane_off = uint32_t((threadIdx.x >> 5) & 3) * 32u << 16;
     const uint32_t tS = tmem + lane_off + C::col_s(q);
     const uint32_t tO = tmem + lane_off + C::col_o(q);
+    const uint32_t tP = tmem + lane_off + C::col_p(q);
     const float sl2 = p.scale_log2;
     const int kc = 1 << p.kc_log2;
-    float m_ref = -INFINITY;  // reference maximum, already scaled to log2 units
+    float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
+    float R_prev = -INFINITY;  // reference that O and l are currently expressed in
     float l = 0.f;
+    int btc = 0, btr = 0;      // window block coordinates of block j
     bool ok = true;
     for (int j = 0; j < w.n_blocks; ++j) {
-        if (__any_sync(0xffffffffu, *abort_flag != 0u)) {
-            ok = false;
-            break;
-        }
         if (!warp_wait(&bars[C::bSFull + q], j & 1, lim)) {
-            record_error(kErrDeviceTimeout);
-            *abort_flag = 1;
             ok = false;
             break;
         }
         sm100::tc_fence_after();
-        uint32_t sa[64], sb[64];
-        sm100::tmem_ld64(tS, sa);
-        sm100::tmem_ld64(tS + 64, sb);
         float s[128];
+        {
+            uint32_t sr[128];
+            sm100::tmem_ld128(tS, sr);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            s[i] = __uint_as_float(sa[i]);
-            s[64 + i] = __uint_as_float(sb[i]);
+            for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
         }
-        // keys of this block that lie outside the window (or past the last
-        // global token) get -inf
+        if (C::kSeparateP) {
+            // S_q may be overwritten by the next block's scores
+            sm100::tc_fence_before();
+            sm100::mbar_arrive(&bars[C::bSFree + q]);
+        }
+        // keys of this block outside the window (or past the last global token) get -inf
         if (j < w.n_win) {
-            const int tr = j / w.wtc, tc = j - tr * w.wtc;
-            const int vc = w.wc1 - (w.wc0 + (tc << p.kc_log2));
-            const int vr = w.wr1 - (w.wr0 + tr * p.kr);
+            const int vc = w.wc1 - (w.wc0 + (btc << p.kc_log2));
+            const int vr = w.wr1 - (w.wr0 + btr * p.kr);
             if (vc < kc || vr < p.kr) {
 #pragma unroll
                 for (int i = 0; i < 128; ++i)
                     if ((i & (kc - 1)) >= vc || (i >> p.kc_log2) >= vr) s[i] = -INFINITY;
+            }
+            if (++btc == w.wtc) {
+                btc = 0;
+                ++btr;
             }
         } else {
             const int vg = p.G - (j - w.n_win) * 128;
@@ -284,17 +434,29 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
                     if (i >= vg) s[i] = -INFINITY;
             }
         }
-        float mx = s[0];
-#pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-        const float m_new = fmaxf(m_ref, mx * sl2);
-        const bool rescale = m_new > m_ref + 8.0f;
-        float alpha = 1.f;
-        if (rescale) {
-            alpha = sm100::ex2_approx(m_ref - m_new);  // 0 on the first block
-            m_ref = m_new;
+        // block maximum and the reference for this block's P (lazy: the
+        // reference moves only when the maximum grows by more than kRescaleLog2)
+        const float bm = row_max128(s) * sl2;
+        if (bm > R + kRescaleLog2) R = bm;
+        // wait for this warpgroup's turn on the exponential unit
+        if ((q == 1 || j > 0) && !warp_wait(&bars[C::bTurn + q], (q == 0 ? j - 1 : j) & 1, lim)) {
+            ok = false;
+            break;
         }
-        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        uint32_t pk[64];
+        const float blk_sum = exp_block(s, sl2, R, pk);
+        __syncwarp();
+        if (lane0) sm100::mbar_arrive(&bars[C::bTurn + (q ^ 1)]);
+        const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
+        if (C::kSeparateP && j > 0) {
+            // PV_q(j-1) must be done before O is rescaled or P_q overwritten
+            if (!warp_wait(&bars[C::bPFree + q], (j - 1) & 1, lim)) {
+                ok = false;
+                break;
+            }
+            sm100::tc_fence_after();
+        }
+        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -304,22 +466,14 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
                 sm100::tmem_st32(tO + c * 32, o);
             }
         }
-        l *= alpha;
-        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-            const float p0 = sm100::ex2_approx(fmaf(s[2 * i], sl2, neg_m));
-            const float p1 = sm100::ex2_approx(fmaf(s[2 * i + 1], sl2, neg_m));
-            l += p0 + p1;
-            pk[i] = sm100::pack_bf16x2(p0, p1);
-        }
-        sm100::tmem_st64(tS, pk);
+        l = l * alpha + blk_sum;
+        sm100::tmem_st64(tP, pk);
         sm100::tc_fence_before();
         sm100::mbar_arrive(&bars[C::bPFull + q]);
+        R_prev = R;
     }
-    if (!ok) return;
-    if (!warp_wait(&bars[C::bOFinal + q], 0, lim)) {
+    if (ok && !warp_wait(&bars[C::bPFree + q], (w.n_blocks - 1) & 1, lim)) ok = false;
+    if (!ok) {
         record_error(kErrDeviceTimeout);
         *abort_flag = 1;
         return;
@@ -357,7 +511,7 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
 // The kernel
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(320, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = KCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = sm100::smem_u32(smem_raw);
@@ -380,10 +534,13 @@ __global__ void __launch_bounds__(320, 1) npa_fwd_kernel(const __grid_constant__
         }
         for (int q = 0; q < 2; ++q) {
             sm100::mbar_init(&bars[C::bSFull + q], 1);
+            sm100::mbar_init(&bars[C::bSFree + q], 128);
             sm100::mbar_init(&bars[C::bPFull + q], 128);
-            sm100::mbar_init(&bars[C::bOFinal + q], 1);
+            sm100::mbar_init(&bars[C::bPFree + q], 1);
+            sm100::mbar_init(&bars[C::bTurn + q], 4);
         }
         sm100::mbar_init(&bars[C::bDrain], 1);
+        sm100::mbar_init(&bars[C::bDrain + 1], 1);
         misc[1] = 0;
         sm100::fence_barrier_init();
     }
@@ -397,11 +554,19 @@ __global__ void __launch_bounds__(320, 1) npa_fwd_kernel(const __grid_constant__
     const uint32_t tmem = misc[0];
     volatile uint32_t *abort_flag = &misc[1];
 
-    if (warp == 8) {
-        if ((threadIdx.x & 31) == 0) run_producer<D>(p, w, smem, bars, abort_flag);
-    } else if (warp == 9) {
-        if ((threadIdx.x & 31) == 0) run_mma<D>(p, w, smem, bars, tmem, abort_flag);
+    if (warp >= 8) {
+        sm100::setmaxnreg_dec<C::kRegsCtl>();
+        if ((threadIdx.x & 31) == 0) {
+            if (warp == 8) run_producer<D>(p, w, smem, bars, abort_flag);
+            if (C::kSeparateP) {
+                if (warp == 9) run_mma_s<D>(p, w, smem, bars, tmem, abort_flag);
+                if (warp == 10) run_mma_pv<D>(p, w, smem, bars, tmem, abort_flag);
+            } else if (warp == 9) {
+                run_mma<D>(p, w, smem, bars, tmem, abort_flag);
+            }
+        }
     } else {
+        sm100::setmaxnreg_inc<C::kRegsSoftmax>();
         run_softmax<D>(p, w, bars, tmem, abort_flag, warp >> 2);
     }
 

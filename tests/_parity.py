@@ -62,6 +62,16 @@ def compare(got: np.ndarray, ref: np.ndarray) -> dict:
     }
 
 
+def log_metrics(name: str, m: dict) -> None:
+    """Appends the comparison to the file named by NPA_PARITY_LOG, if set."""
+    import json
+    import os
+    path = os.environ.get("NPA_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": name, **m}) + "\n")
+
+
 def passes(m: dict) -> bool:
     return m["finite"] and m["max_abs"] <= MAX_ABS and m["mean_abs"] <= MEAN_ABS and m["rel_l2"] <= REL_L2
 

@@ -14,7 +14,7 @@ import pytest
 
 import oracle
 from workloads import PRESETS, Workload, make_inputs, f64_to_bf16_bits
-from _parity import compare, passes, run_gpu, run_oracle, sample_queries, to_device, to_f64
+from _parity import compare, log_metrics, passes, run_gpu, run_oracle, sample_queries, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -59,6 +59,7 @@ def test_small_full_parity(w):
     got = to_f64(run_gpu(w, inp))
     ref = run_oracle(w, inp)
     m = compare(got, ref)
+    log_metrics(w.name, m)
     assert passes(m), m
 
 
@@ -74,6 +75,7 @@ def test_full_workload_sampled_parity(name):
     idx = torch.from_numpy(((qs[:, 0].astype(np.int64) * w.heads + qs[:, 1]) * (w.H * w.W) + qs[:, 2])).cuda()
     got = to_f64(flat.index_select(0, idx))
     m = compare(got, ref)
+    log_metrics(name + " (sampled)", m)
     assert passes(m), m
     # every output row was written (the buffer starts as NaN)
     assert bool(torch.isfinite(o).all())
