@@ -43,7 +43,7 @@ KERNEL_NAME = "npa_fwd_kernel"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(PRESETS))
@@ -203,7 +203,7 @@ class ClockSampler:
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -321,35 +321,63 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     value = world * flops * args.steps / (timed_ms * 1e-3) / 1e12
     avg_kernel_ms = kernel_ms_sum / args.steps
 
-    # end to end through host buffers: H2D of the inputs, the call, D2H of O
+    # End to end through host buffers: every step copies its inputs from pinned
+    # host memory, runs the call and reads the output back. Steps are pipelined
+    # over three streams with double-buffered device tensors, so step i+1's
+    # upload overlaps step i's kernel and step i-1's download.
     e2e = None
     if not args.no_e2e:
         hq, hk, hv = (x.to("cpu").pin_memory() for x in (q, k, v))
         hg = [x.to("cpu").pin_memory() for x in (gk, gv)] if w.G else []
-        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hos = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for _ in range(2)]
+        bufs = [(q, k, v, gk, gv, o)]
+        bufs.append(tuple(torch.empty_like(x) if x is not None else None for x in (q, k, v, gk, gv, o)))
         h2d = sum(x.numel() * 2 for x in [hq, hk, hv] + hg)
-        d2h = ho.numel() * 2
+        d2h = o.numel() * 2
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_k = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            if w.G:
-                gk.copy_(hg[0], non_blocking=True)
-                gv.copy_(hg[1], non_blocking=True)
-            call()
-            ho.copy_(o, non_blocking=True)
+        def e2e_steps(n):
+            for i in range(n):
+                b = i % 2
+                bq, bk, bv, bgk, bgv, bo = bufs[b]
+                with torch.cuda.stream(s_in):
+                    if i >= 2:
+                        s_in.wait_event(ev_k[b])
+                    bq.copy_(hq, non_blocking=True)
+                    bk.copy_(hk, non_blocking=True)
+                    bv.copy_(hv, non_blocking=True)
+                    if w.G:
+                        bgk.copy_(hg[0], non_blocking=True)
+                        bgv.copy_(hg[1], non_blocking=True)
+                    ev_in[b].record(s_in)
+                stream.wait_event(ev_in[b])
+                if i >= 2:
+                    stream.wait_event(ev_out[b])
+                if w.geometry == "npa":
+                    npa.npa_attention_fwd(bq, bk, bv, bo, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, bgk, bgv,
+                                          w.G, stream)
+                else:
+                    npa.pcpp_attention_fwd(bq, bk, bv, bo, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, bgk,
+                                           bgv, w.G, stream)
+                ev_k[b].record(stream)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(ev_k[b])
+                    hos[b].copy_(bo, non_blocking=True)
+                    ev_out[b].record(s_out)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        e2e_steps(max(2, args.warmup))
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        e2e_steps(args.steps)
+        s_out.wait_stream(stream)
+        s_out.wait_stream(s_in)
+        e1.record(s_out)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
         if world > 1:
@@ -357,7 +385,11 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
         e2e = {"value": world * flops * args.steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps,
+               "pipelined": "upload / kernel / download on three streams, double-buffered"}
+        status = npa.npa_device_status(stream)
+        if status != npa.NPA_OK:
+            raise RuntimeError(f"device status {npa.npa_status_string(status)}")
 
     if rank != 0:
         return

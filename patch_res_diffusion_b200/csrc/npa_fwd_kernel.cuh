@@ -354,6 +354,39 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
     return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
 }
 
+// Fraction (in eighths) of the exponentials evaluated on the FMA pipe. Off
+// by default: measured on B200 at d = 64, every fraction from 2/8 to 5/8 made
+// the kernel slower (the exponential phase is limited by instruction issue
+// and latency as much as by the special-function unit's throughput).
+#ifndef NPA_EXP_EMU8
+#define NPA_EXP_EMU8 0
+#endif
+
+// 2^x for a pair of arguments without the special-function unit: Cody-Waite
+// reduction x = j + f, j = round(x) by the float32 magic-number addition
+// (1.5 * 2^23), f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial
+// (relative error 7.5e-5, fitted by fit_exp2_poly.py); 2^j added to the
+// exponent field. Arguments below -125 (masked keys: -inf) give exactly 0.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float &p0, float &p1) {
+    float x0, x1;
+    sm100::unpack_f32x2(x2, x0, x1);
+    const uint64_t xc = sm100::pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t magic = sm100::pack_f32x2(12582912.f, 12582912.f);
+    const uint64_t neg_magic = sm100::pack_f32x2(-12582912.f, -12582912.f);
+    const uint64_t t = sm100::add_f32x2(xc, magic);
+    const uint64_t jn = sm100::add_f32x2(neg_magic, t);                        // j
+    const uint64_t f = sm100::fma_f32x2(jn, sm100::pack_f32x2(-1.f, -1.f), xc);  // x - j
+    uint64_t p = sm100::fma_f32x2(sm100::pack_f32x2(0.0551716685295105f, 0.0551716685295105f), f,
+                                  sm100::pack_f32x2(0.2426111251115799f, 0.2426111251115799f));
+    p = sm100::fma_f32x2(p, f, sm100::pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
+    p = sm100::fma_f32x2(p, f, sm100::pack_f32x2(0.9999280571937561f, 0.9999280571937561f));
+    float q0, q1, t0, t1;
+    sm100::unpack_f32x2(p, q0, q1);
+    sm100::unpack_f32x2(t, t0, t1);
+    p0 = x0 < -125.f ? 0.f : __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    p1 = x1 < -125.f ? 0.f : __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // p = 2^(s*c - ref) for 128 scores: packed bf16 pairs into pk, float32 sum returned.
 __device__ __forceinline__ float exp_block(const float (&s)[128], float c, float ref, uint32_t (&pk)[64]) {
     const float neg = (ref == -INFINITY) ? 0.f : -ref;
@@ -363,9 +396,15 @@ __device__ __forceinline__ float exp_block(const float (&s)[128], float c, float
 #pragma unroll
     for (int i = 0; i < 64; ++i) {
         const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
-        float x0, x1;
-        sm100::unpack_f32x2(x2, x0, x1);
-        const float p0 = sm100::ex2_approx(x0), p1 = sm100::ex2_approx(x1);
+        float p0, p1;
+        if ((i & 7) < NPA_EXP_EMU8) {
+            exp2_poly_x2(x2, p0, p1);
+        } else {
+            float x0, x1;
+            sm100::unpack_f32x2(x2, x0, x1);
+            p0 = sm100::ex2_approx(x0);
+            p1 = sm100::ex2_approx(x1);
+        }
         pk[i] = sm100::pack_bf16x2(p0, p1);
         acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
     }
