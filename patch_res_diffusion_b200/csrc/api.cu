@@ -31,12 +31,14 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
     bool checked = false;
     npa_status status = NPA_ERR_UNSUPPORTED;
+    int sm_count = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
 // Resolves the tensor-map encoder and checks (once per device) that the
 // current device is an sm_100 part; sets the kernels' shared-memory limits.
-npa_status ensure_ready() {
+// On success *sm_count holds the device's multiprocessor count.
+npa_status ensure_ready(int *sm_count = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NPA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return NPA_ERR_UNSUPPORTED;
@@ -55,6 +57,9 @@ npa_status ensure_ready() {
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NPA_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            ds.sm_count < 1)
+            return NPA_ERR_CUDA;
         if (major != 10 || minor != 0) {
             ds.status = NPA_ERR_UNSUPPORTED;
         } else if (cudaFuncSetAttribute(npa::npa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -67,6 +72,7 @@ npa_status ensure_ready() {
         }
         ds.checked = true;
     }
+    if (sm_count) *sm_count = ds.sm_count;
     return ds.status;
 }
 
@@ -182,9 +188,43 @@ npa_status validate_common(const void *q, const void *k, const void *v, void *o,
     return NPA_OK;
 }
 
+// Patches ordered by decreasing number of key blocks (ties: natural order),
+// so a persistent CTA's last units are its cheapest.
+void order_patches(const Geo &g, FwdParams &prm) {
+    const int np = prm.nPh * prm.nPw;
+    if (np > npa::kMaxPatchOrder) {
+        prm.n_perm = 0;
+        return;
+    }
+    const int kc = 1 << prm.kc_log2;
+    int cost[npa::kMaxPatchOrder];
+    for (int pi = 0; pi < prm.nPh; ++pi) {
+        for (int pj = 0; pj < prm.nPw; ++pj) {
+            const int r0 = pi * g.Ph, r1 = r0 + g.Ph < g.H ? r0 + g.Ph : g.H;
+            const int c0 = pj * g.Pw, c1 = c0 + g.Pw < g.W ? c0 + g.Pw : g.W;
+            const int wh = (r1 + g.mh < g.H ? r1 + g.mh : g.H) - (r0 - g.mh > 0 ? r0 - g.mh : 0);
+            const int ww = (c1 + g.mw < g.W ? c1 + g.mw : g.W) - (c0 - g.mw > 0 ? c0 - g.mw : 0);
+            cost[pi * prm.nPw + pj] = ((ww + kc - 1) / kc) * ((wh + prm.kr - 1) / prm.kr);
+        }
+    }
+    for (int i = 0; i < np; ++i) prm.patch_order[i] = (unsigned short)i;
+    // insertion sort, stable, descending cost (np <= 256)
+    for (int i = 1; i < np; ++i) {
+        const unsigned short x = prm.patch_order[i];
+        int j = i - 1;
+        while (j >= 0 && cost[prm.patch_order[j]] < cost[x]) {
+            prm.patch_order[j + 1] = prm.patch_order[j];
+            --j;
+        }
+        prm.patch_order[j + 1] = x;
+    }
+    prm.n_perm = np;
+}
+
 npa_status launch(const void *q, const void *k, const void *v, void *o, int B, int heads, int d, const Geo &g,
                   int G, const npa_global_kv *gkv, npa_stream_t stream) {
-    npa_status st = ensure_ready();
+    int sm_count = 0;
+    npa_status st = ensure_ready(&sm_count);
     if (st != NPA_OK) return st;
 
     FwdParams prm;
@@ -209,9 +249,15 @@ npa_status launch(const void *q, const void *k, const void *v, void *o, int B, i
     prm.wait_limit_ns = kWaitLimitNs;
 
     const long long units = (long long)B * heads * prm.nPh * prm.nPw * prm.n_qblocks;
-    if (units > INT_MAX || (long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
+    if (units > INT_MAX / 2 || (long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
 
     const int BH = B * heads;
+    prm.BH = BH;
+    prm.n_units = (int)units;
+    order_patches(g, prm);
+    // persistent grid: one CTA per multiprocessor (shared memory and TMEM
+    // admit one), each walking every gridDim.x-th unit
+    const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)BH};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)g.W * d * 2, (cuuint64_t)g.H * g.W * d * 2};
     const cuuint32_t qbox[4] = {64, (cuuint32_t)prm.qc, (cuuint32_t)prm.qr, 1};
@@ -231,10 +277,10 @@ npa_status launch(const void *q, const void *k, const void *v, void *o, int B, i
     void *args[1] = {&prm};
     cudaError_t e;
     if (d == 64)
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3((unsigned)units), dim3(npa::KCfg<64>::kThreads), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3(grid), dim3(npa::KCfg<64>::kThreads), args,
                              npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
     else
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3((unsigned)units), dim3(npa::KCfg<128>::kThreads), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3(grid), dim3(npa::KCfg<128>::kThreads), args,
                              npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
     return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
 }

@@ -82,7 +82,8 @@ struct KCfg {
     static constexpr int kOffBar = kOffV + kStages * kTileBytes;
     // barrier indices
     static constexpr int bQFull = 0;
-    static constexpr int bKFull = 1;
+    static constexpr int bQEmpty = 1;                  // Q buffer free (S issuer commit after a unit)
+    static constexpr int bKFull = 2;
     static constexpr int bKEmpty = bKFull + kStages;
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
@@ -102,6 +103,17 @@ struct KCfg {
     __device__ static constexpr uint32_t col_o(int q) { return 256u + (q ? uint32_t(D) : 0u); }
     __device__ static constexpr uint32_t col_p(int q) { return kSeparateP ? (384u + (q ? 64u : 0u)) : col_s(q); }
 };
+
+// ---------------------------------------------------------------------------
+// Persistent work loop. Every role of a CTA walks the same unit sequence
+// (blockIdx.x, blockIdx.x + gridDim.x, ...) and skips the same empty units, so
+// the roles agree on every barrier phase without exchanging unit indices.
+// Phases are counted across units: gb = key blocks processed so far by this
+// CTA (one S and one P per tile per block), uq = units processed so far.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool unit_has_work(const FwdParams &p, const Work &w) {
+    return q_tile_valid(p, w, w.tile0) || q_tile_valid(p, w, w.tile0 + 1);
+}
 
 // ---------------------------------------------------------------------------
 // Producer: one thread of warp 8.
@@ -127,8 +139,7 @@ __device__ __forceinline__ void load_block(const FwdParams &p, const Work &w, in
 }
 
 template <int D>
-__device__ void run_producer(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars,
-                             volatile uint32_t *abort_flag) {
+__device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     sm100::tma_prefetch_desc(&p.tm_q);
@@ -139,40 +150,56 @@ __device__ void run_producer(const FwdParams &p, const Work &w, uint8_t *smem, u
         sm100::tma_prefetch_desc(&p.tm_gv);
     }
     const uint32_t q_bytes = uint32_t(C::kChunks * p.qc * p.qr * 128);
-    sm100::mbar_arrive_expect_tx(&bars[C::bQFull], 2 * q_bytes);
+    int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q pairs issued
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+        const Work w = decode_work(p, unit);
+        if (!unit_has_work(p, w)) continue;
+        // the previous unit's last S products must be done with the Q buffer
+        if (uq > 0 && !sm100::mbar_wait(&bars[C::bQEmpty], (uq - 1) & 1, lim)) {
+            ok = false;
+            break;
+        }
+        sm100::mbar_arrive_expect_tx(&bars[C::bQFull], 2 * q_bytes);
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        int row0, col0;
-        q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
+        for (int t = 0; t < 2; ++t) {
+            int row0, col0;
+            q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
-                               &bars[C::bQFull], c * 64, col0, row0, w.bh);
+            for (int c = 0; c < C::kChunks; ++c)
+                sm100::tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                                   &bars[C::bQFull], c * 64, col0, row0, w.bh);
+        }
+        ++uq;
+        for (int j = 0; j < w.n_blocks; ++j) {
+            if (*abort_flag) {
+                ok = false;
+                break;
+            }
+            const int s = nk % C::kStages, use = nk / C::kStages;
+            if (use > 0 && !sm100::mbar_wait(&bars[C::bKEmpty + s], (use - 1) & 1, lim)) {
+                ok = false;
+                break;
+            }
+            sm100::mbar_arrive_expect_tx(&bars[C::bKFull + s], C::kTileBytes);
+            load_block<D>(p, w, j, false, smem + C::kOffK + s * C::kTileBytes, &bars[C::bKFull + s]);
+            ++nk;
+            if (use > 0 && !sm100::mbar_wait(&bars[C::bVEmpty + s], (use - 1) & 1, lim)) {
+                ok = false;
+                break;
+            }
+            sm100::mbar_arrive_expect_tx(&bars[C::bVFull + s], C::kTileBytes);
+            load_block<D>(p, w, j, true, smem + C::kOffV + s * C::kTileBytes, &bars[C::bVFull + s]);
+            ++nv;
+        }
     }
-    int nk = 0, nv = 0;  // K / V blocks issued
-    for (int j = 0; j < w.n_blocks; ++j) {
-        if (*abort_flag) break;
-        const int s = j % C::kStages, use = j / C::kStages;
-        if (use > 0 && !sm100::mbar_wait(&bars[C::bKEmpty + s], (use - 1) & 1, lim)) {
-            record_error(kErrDeviceTimeout);
-            *abort_flag = 1;
-            break;
-        }
-        sm100::mbar_arrive_expect_tx(&bars[C::bKFull + s], C::kTileBytes);
-        load_block<D>(p, w, j, false, smem + C::kOffK + s * C::kTileBytes, &bars[C::bKFull + s]);
-        ++nk;
-        if (use > 0 && !sm100::mbar_wait(&bars[C::bVEmpty + s], (use - 1) & 1, lim)) {
-            record_error(kErrDeviceTimeout);
-            *abort_flag = 1;
-            break;
-        }
-        sm100::mbar_arrive_expect_tx(&bars[C::bVFull + s], C::kTileBytes);
-        load_block<D>(p, w, j, true, smem + C::kOffV + s * C::kTileBytes, &bars[C::bVFull + s]);
-        ++nv;
+    if (!ok) {
+        record_error(kErrDeviceTimeout);
+        *abort_flag = 1;
     }
     // Drain: every issued copy must have landed before the CTA may exit
     // (immediate on the normal path, where the consumers already saw them).
-    sm100::mbar_wait(&bars[C::bQFull], 0, lim);
+    if (uq > 0) sm100::mbar_wait(&bars[C::bQFull], (uq - 1) & 1, lim);
     for (int s = 0; s < C::kStages; ++s) {
         if (nk > s) sm100::mbar_wait(&bars[C::bKFull + s], ((nk - 1 - s) / C::kStages) & 1, lim);
         if (nv > s) sm100::mbar_wait(&bars[C::bVFull + s], ((nv - 1 - s) / C::kStages) & 1, lim);
@@ -180,7 +207,7 @@ __device__ void run_producer(const FwdParams &p, const Work &w, uint8_t *smem, u
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer: one thread of warp 9.
+// MMA issuers
 // ---------------------------------------------------------------------------
 // Shared-memory descriptors are built once per operand buffer; stepping
 // through K (16 elements = 32 bytes inside a 128-byte swizzle atom, or the
@@ -229,26 +256,38 @@ __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
 // d = 64 (P has its own TMEM buffer): the S products and the P.V products
 // touch disjoint tensor memory and shared memory, so two warps issue them
 // independently. This one issues S_0(j), S_1(j) as soon as the softmax warps
-// hold S(j-1) in registers.
+// hold S(j-1) in registers; the first S of a unit also overlaps the previous
+// unit's last P.V products and epilogue.
 template <int D>
-__device__ void run_mma_s(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+__device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                           volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     const OperandDescs dd = make_descs<D>(smem);
-    bool ok = sm100::mbar_wait(&bars[C::bQFull], 0, lim);
-    for (int j = 0; ok && j < w.n_blocks; ++j) {
-        if (*abort_flag) break;
-        const int s = j % C::kStages;
-        ok = sm100::mbar_wait(&bars[C::bKFull + s], (j / C::kStages) & 1, lim);
-        for (int q = 0; ok && q < 2; ++q) {
-            if (j > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (j - 1) & 1, lim);
-            if (!ok) break;
-            sm100::tc_fence_after();
-            issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + s * dd.stage);
-            sm100::tc_commit(&bars[C::bSFull + q]);
+    int gb = 0, uq = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+        const Work w = decode_work(p, unit);
+        if (!unit_has_work(p, w)) continue;
+        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
+        ++uq;
+        for (int j = 0; ok && j < w.n_blocks; ++j, ++gb) {
+            if (*abort_flag) {
+                ok = false;
+                break;
+            }
+            const int s = gb % C::kStages;
+            ok = sm100::mbar_wait(&bars[C::bKFull + s], (gb / C::kStages) & 1, lim);
+            for (int q = 0; ok && q < 2; ++q) {
+                if (gb > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (gb - 1) & 1, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + s * dd.stage);
+                sm100::tc_commit(&bars[C::bSFull + q]);
+            }
+            if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
         }
-        if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
+        if (ok) sm100::tc_commit(&bars[C::bQEmpty]);  // this unit's Q is no longer read
     }
     if (!ok) {
         record_error(kErrDeviceTimeout);
@@ -260,24 +299,32 @@ __device__ void run_mma_s(const FwdParams &p, const Work &w, uint8_t *smem, uint
 
 // d = 64: the P.V products, O_q(j) += P_q(j) V(j) as each P_q(j) arrives.
 template <int D>
-__device__ void run_mma_pv(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+__device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                            volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     const OperandDescs dd = make_descs<D>(smem);
+    int gb = 0;
     bool ok = true;
-    for (int j = 0; ok && j < w.n_blocks; ++j) {
-        if (*abort_flag) break;
-        const int s = j % C::kStages;
-        ok = sm100::mbar_wait(&bars[C::bVFull + s], (j / C::kStages) & 1, lim);
-        for (int q = 0; ok && q < 2; ++q) {
-            ok = sm100::mbar_wait(&bars[C::bPFull + q], j & 1, lim);
-            if (!ok) break;
-            sm100::tc_fence_after();
-            issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > 0);
-            sm100::tc_commit(&bars[C::bPFree + q]);
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+        const Work w = decode_work(p, unit);
+        if (!unit_has_work(p, w)) continue;
+        for (int j = 0; ok && j < w.n_blocks; ++j, ++gb) {
+            if (*abort_flag) {
+                ok = false;
+                break;
+            }
+            const int s = gb % C::kStages;
+            ok = sm100::mbar_wait(&bars[C::bVFull + s], (gb / C::kStages) & 1, lim);
+            for (int q = 0; ok && q < 2; ++q) {
+                ok = sm100::mbar_wait(&bars[C::bPFull + q], gb & 1, lim);
+                if (!ok) break;
+                sm100::tc_fence_after();
+                issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > 0);
+                sm100::tc_commit(&bars[C::bPFree + q]);
+            }
+            if (ok) sm100::tc_commit(&bars[C::bVEmpty + s]);
         }
-        if (ok) sm100::tc_commit(&bars[C::bVEmpty + s]);
     }
     if (!ok) {
         record_error(kErrDeviceTimeout);
@@ -290,40 +337,54 @@ __device__ void run_mma_pv(const FwdParams &p, const Work &w, uint8_t *smem, uin
 // d = 128 (P aliases S): one warp issues everything, PV_q(j-1) before S_q(j)
 // for each tile, so that the completion of S_q(j) also implies PV_q(j-1).
 template <int D>
-__device__ void run_mma(const FwdParams &p, const Work &w, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+__device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                         volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     const OperandDescs dd = make_descs<D>(smem);
-    const int n = w.n_blocks;
-    bool ok = sm100::mbar_wait(&bars[C::bQFull], 0, lim);
-    for (int j = 0; ok && j <= n; ++j) {
-        if (*abort_flag) break;
-        if (j < n) {
-            ok = sm100::mbar_wait(&bars[C::bKFull + j % C::kStages], (j / C::kStages) & 1, lim);
-            if (!ok) break;
-        }
-        if (j > 0) {
-            ok = sm100::mbar_wait(&bars[C::bVFull + (j - 1) % C::kStages], ((j - 1) / C::kStages) & 1, lim);
-            if (!ok) break;
-        }
+    int gb = 0, uq = 0;  // gb: global index of block j = 0 of the current unit
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+        const Work w = decode_work(p, unit);
+        if (!unit_has_work(p, w)) continue;
+        const int n = w.n_blocks;
+        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
+        ++uq;
         sm100::tc_fence_after();
-        for (int q = 0; q < 2; ++q) {
-            if (j > 0) {
-                ok = sm100::mbar_wait(&bars[C::bPFull + q], (j - 1) & 1, lim);
-                if (!ok) break;
-                sm100::tc_fence_after();
-                issue_pv<D>(tmem, q, dd.v0 + ((j - 1) % C::kStages) * dd.stage, j > 1);
-                sm100::tc_commit(&bars[C::bPFree + q]);
+        for (int j = 0; ok && j <= n; ++j) {
+            if (*abort_flag) {
+                ok = false;
+                break;
             }
+            const int g = gb + j;  // global index of block j
             if (j < n) {
-                issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + (j % C::kStages) * dd.stage);
-                sm100::tc_commit(&bars[C::bSFull + q]);
+                ok = sm100::mbar_wait(&bars[C::bKFull + g % C::kStages], (g / C::kStages) & 1, lim);
+                if (!ok) break;
             }
+            if (j > 0) {
+                ok = sm100::mbar_wait(&bars[C::bVFull + (g - 1) % C::kStages], ((g - 1) / C::kStages) & 1, lim);
+                if (!ok) break;
+            }
+            sm100::tc_fence_after();
+            for (int q = 0; q < 2; ++q) {
+                if (j > 0) {
+                    ok = sm100::mbar_wait(&bars[C::bPFull + q], (g - 1) & 1, lim);
+                    if (!ok) break;
+                    sm100::tc_fence_after();
+                    issue_pv<D>(tmem, q, dd.v0 + ((g - 1) % C::kStages) * dd.stage, j > 1);
+                    sm100::tc_commit(&bars[C::bPFree + q]);
+                }
+                if (j < n) {
+                    issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + (g % C::kStages) * dd.stage);
+                    sm100::tc_commit(&bars[C::bSFull + q]);
+                }
+            }
+            if (!ok) break;
+            if (j < n) sm100::tc_commit(&bars[C::bKEmpty + g % C::kStages]);
+            if (j == n - 1) sm100::tc_commit(&bars[C::bQEmpty]);
+            if (j > 0) sm100::tc_commit(&bars[C::bVEmpty + (g - 1) % C::kStages]);
         }
-        if (!ok) break;
-        if (j < n) sm100::tc_commit(&bars[C::bKEmpty + j % C::kStages]);
-        if (j > 0) sm100::tc_commit(&bars[C::bVEmpty + (j - 1) % C::kStages]);
+        gb += n;
     }
     if (!ok) {
         record_error(kErrDeviceTimeout);
@@ -417,8 +478,8 @@ __device__ __forceinline__ float exp_block(const float (&s)[128], float c, float
 }
 
 template <int D>
-__device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, uint32_t tmem,
-                            volatile uint32_t *abort_flag, int q) {
+__device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
+                            int q) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
     const int row = threadIdx.x & 127;
@@ -429,13 +490,17 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
     const uint32_t tP = tmem + lane_off + C::col_p(q);
     const float sl2 = p.scale_log2;
     const int kc = 1 << p.kc_log2;
+    int gb = 0;  // global index (across units) of the current block
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    const Work w = decode_work(p, unit);
+    if (!unit_has_work(p, w)) continue;
     float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
     float R_prev = -INFINITY;  // reference that O and l are currently expressed in
     float l = 0.f;
     int btc = 0, btr = 0;      // window block coordinates of block j
-    bool ok = true;
-    for (int j = 0; j < w.n_blocks; ++j) {
-        if (!warp_wait(&bars[C::bSFull + q], j & 1, lim)) {
+    for (int j = 0; j < w.n_blocks; ++j, ++gb) {
+        if (!warp_wait(&bars[C::bSFull + q], gb & 1, lim)) {
             ok = false;
             break;
         }
@@ -478,7 +543,7 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
         const float bm = row_max128(s) * sl2;
         if (bm > R + kRescaleLog2) R = bm;
         // wait for this warpgroup's turn on the exponential unit
-        if ((q == 1 || j > 0) && !warp_wait(&bars[C::bTurn + q], (q == 0 ? j - 1 : j) & 1, lim)) {
+        if ((q == 1 || gb > 0) && !warp_wait(&bars[C::bTurn + q], (q == 0 ? gb - 1 : gb) & 1, lim)) {
             ok = false;
             break;
         }
@@ -489,7 +554,7 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
         if (C::kSeparateP && j > 0) {
             // PV_q(j-1) must be done before O is rescaled or P_q overwritten
-            if (!warp_wait(&bars[C::bPFree + q], (j - 1) & 1, lim)) {
+            if (!warp_wait(&bars[C::bPFree + q], (gb - 1) & 1, lim)) {
                 ok = false;
                 break;
             }
@@ -511,12 +576,9 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
         sm100::mbar_arrive(&bars[C::bPFull + q]);
         R_prev = R;
     }
-    if (ok && !warp_wait(&bars[C::bPFree + q], (w.n_blocks - 1) & 1, lim)) ok = false;
-    if (!ok) {
-        record_error(kErrDeviceTimeout);
-        *abort_flag = 1;
-        return;
-    }
+    // the last PV of this tile completes phase gb-1 of P_free
+    if (ok && !warp_wait(&bars[C::bPFree + q], (gb - 1) & 1, lim)) ok = false;
+    if (!ok) break;
     sm100::tc_fence_after();
     // epilogue: O / l -> bf16 -> the query's token position
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
@@ -544,6 +606,11 @@ __device__ void run_softmax(const FwdParams &p, const Work &w, uint64_t *bars, u
             }
         }
     }
+    }
+    if (!ok) {
+        record_error(kErrDeviceTimeout);
+        *abort_flag = 1;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -556,15 +623,13 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
     const uint32_t raw = sm100::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
 
-    const Work w = decode_work(p, blockIdx.x);
-    if (!q_tile_valid(p, w, w.tile0) && !q_tile_valid(p, w, w.tile0 + 1)) return;
-
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);  // [0] TMEM base, [1] abort flag
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
         sm100::mbar_init(&bars[C::bQFull], 1);
+        sm100::mbar_init(&bars[C::bQEmpty], 1);
         for (int s = 0; s < C::kStages; ++s) {
             sm100::mbar_init(&bars[C::bKFull + s], 1);
             sm100::mbar_init(&bars[C::bKEmpty + s], 1);
@@ -596,17 +661,17 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
     if (warp >= 8) {
         sm100::setmaxnreg_dec<C::kRegsCtl>();
         if ((threadIdx.x & 31) == 0) {
-            if (warp == 8) run_producer<D>(p, w, smem, bars, abort_flag);
+            if (warp == 8) run_producer<D>(p, smem, bars, abort_flag);
             if (C::kSeparateP) {
-                if (warp == 9) run_mma_s<D>(p, w, smem, bars, tmem, abort_flag);
-                if (warp == 10) run_mma_pv<D>(p, w, smem, bars, tmem, abort_flag);
+                if (warp == 9) run_mma_s<D>(p, smem, bars, tmem, abort_flag);
+                if (warp == 10) run_mma_pv<D>(p, smem, bars, tmem, abort_flag);
             } else if (warp == 9) {
-                run_mma<D>(p, w, smem, bars, tmem, abort_flag);
+                run_mma<D>(p, smem, bars, tmem, abort_flag);
             }
         }
     } else {
         sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D>(p, w, bars, tmem, abort_flag, warp >> 2);
+        run_softmax<D>(p, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();

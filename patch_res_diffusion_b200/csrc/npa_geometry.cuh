@@ -10,7 +10,8 @@
 //     window of strip i is rows [i*s - r, (i+1)*s + r) clipped, all columns:
 //     the strip plus the r adjacent rows of each neighbouring strip.
 //
-// Work unit = (batch*head, patch, pair of 128-row query tiles). A query tile is
+// Work unit = (batch*head, patch, pair of 128-row query tiles); a persistent
+// CTA walks the units blockIdx.x, blockIdx.x + gridDim.x, ... A query tile is
 // a box of qr patch rows x qc patch columns (qr*qc <= 128); a key/value block
 // is a box of kr rows x kc columns (kr*kc = 128) inside the window, followed
 // by ceil(G/128) blocks of global tokens. Every quantity is recomputed from
@@ -21,6 +22,10 @@
 #include <cuda.h>
 
 namespace npa {
+
+// Up to this many patches are visited largest window first; beyond it, in
+// natural order.
+constexpr int kMaxPatchOrder = 256;
 
 struct FwdParams {
     CUtensorMap tm_q;   // 4D {d, W, H, B*heads}, box {64, qc, qr, 1}, 128B swizzle
@@ -37,6 +42,10 @@ struct FwdParams {
     int n_qblocks;                   // query-tile pairs per patch
     float scale_log2;                // log2(e) / sqrt(d)
     unsigned long long wait_limit_ns;
+    int BH;                          // batch * heads
+    int n_units;                     // work units in execution order
+    int n_perm;                      // entries of patch_order (0: natural order)
+    unsigned short patch_order[kMaxPatchOrder];  // patches by decreasing window area
 };
 
 struct Work {
@@ -52,13 +61,16 @@ __host__ __device__ inline int imin_(int a, int b) { return a < b ? a : b; }
 __host__ __device__ inline int imax_(int a, int b) { return a > b ? a : b; }
 __host__ __device__ inline int cdiv_(int a, int b) { return (a + b - 1) / b; }
 
+// Work units are ordered query-tile pair fastest, then batch*head, then
+// patch (largest window first), so the units that run at the same time share
+// few key/value windows (they stay in L2) and the cheapest units come last.
 __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     Work w;
     const int qb = unit % p.n_qblocks;
     const int rest = unit / p.n_qblocks;
-    const int np = p.nPh * p.nPw;
-    const int patch = rest % np;
-    w.bh = rest / np;
+    w.bh = rest % p.BH;
+    const int rank = rest / p.BH;
+    const int patch = rank < p.n_perm ? int(p.patch_order[rank]) : rank;
     const int pi = patch / p.nPw, pj = patch % p.nPw;
     w.pr0 = pi * p.Ph;
     w.pr1 = imin_(p.H, w.pr0 + p.Ph);
