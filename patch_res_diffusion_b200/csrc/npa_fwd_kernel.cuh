@@ -99,6 +99,10 @@ struct KCfg {
     // tensor memory columns
     static constexpr uint32_t kTmemCols = 512;
     static constexpr bool kSeparateP = (D == 64);
+    // d = 64: the softmax warpgroups hand the exponential unit to each other
+    // (measured +5..7%); d = 128: the aliased-P issue order already alternates
+    // the tiles and the hand-off costs about 3%.
+    static constexpr bool kUseTurn = (D == 64);
     __device__ static constexpr uint32_t col_s(int q) { return q ? 128u : 0u; }
     __device__ static constexpr uint32_t col_o(int q) { return 256u + (q ? uint32_t(D) : 0u); }
     __device__ static constexpr uint32_t col_p(int q) { return kSeparateP ? (384u + (q ? 64u : 0u)) : col_s(q); }
@@ -543,14 +547,17 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         const float bm = row_max128(s) * sl2;
         if (bm > R + kRescaleLog2) R = bm;
         // wait for this warpgroup's turn on the exponential unit
-        if ((q == 1 || gb > 0) && !warp_wait(&bars[C::bTurn + q], (q == 0 ? gb - 1 : gb) & 1, lim)) {
+        if (C::kUseTurn && (q == 1 || gb > 0) &&
+            !warp_wait(&bars[C::bTurn + q], (q == 0 ? gb - 1 : gb) & 1, lim)) {
             ok = false;
             break;
         }
         uint32_t pk[64];
         const float blk_sum = exp_block(s, sl2, R, pk);
-        __syncwarp();
-        if (lane0) sm100::mbar_arrive(&bars[C::bTurn + (q ^ 1)]);
+        if (C::kUseTurn) {
+            __syncwarp();
+            if (lane0) sm100::mbar_arrive(&bars[C::bTurn + (q ^ 1)]);
+        }
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
         if (C::kSeparateP && j > 0) {
             // PV_q(j-1) must be done before O is rescaled or P_q overwritten
