@@ -34,8 +34,8 @@ from . import build as _build
 
 __all__ = [
     "lib", "npa_key_set", "pcpp_key_set", "pcpp_neighbor_rows", "npa_attention",
-    "pcpp_attention", "pair_count", "num_threads", "dense_mask", "dense_attention",
-    "bf16_to_f64",
+    "pcpp_attention", "pcpp_attention_stale", "pair_count", "num_threads", "dense_mask",
+    "dense_attention", "dense_pcpp_stale", "bf16_to_f64",
 ]
 
 _LIB = None
@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_pcpp_attention.argtypes = common + [ctypes.c_int, ctypes.c_double, ctypes.c_int,
                                                      ctypes.c_void_p, ctypes.c_long]
         L.oracle_pcpp_attention.restype = ctypes.c_int
+        L.oracle_pcpp_attention_stale.argtypes = [u16p] * 7 + [ctypes.c_void_p] + [ctypes.c_int] * 5 + [
+            ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_long]
+        L.oracle_pcpp_attention_stale.restype = ctypes.c_int
         L.oracle_pair_count.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
         L.oracle_pair_count.restype = ctypes.c_longlong
         L.oracle_num_threads.argtypes = []
@@ -153,6 +156,32 @@ def pcpp_attention(q, k, v, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None,
                  W, d, G, queries)
 
 
+def pcpp_attention_stale(q, k, v, ks, vs, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None, G=0,
+                         queries: Optional[Sequence] = None) -> np.ndarray:
+    """PCPP attention with stale neighbour rows, float64: the keys of a query's
+    own strip come from k/v, the borrowed neighbour rows from ks/vs (the
+    previous step's keys/values, same layout)."""
+    q, qp = _u16(q)
+    k, kp = _u16(k)
+    v, vp = _u16(v)
+    ks, ksp = _u16(ks)
+    vs, vsp = _u16(vs)
+    gk, gkp = _u16(gk)
+    gv, gvp = _u16(gv)
+    if queries is None:
+        out = np.empty((B, heads, H * W, d), dtype=np.float64)
+        qs_p, nq = None, 0
+    else:
+        qs = np.ascontiguousarray(np.asarray(queries, dtype=np.int32).reshape(-1, 3))
+        out = np.empty((qs.shape[0], d), dtype=np.float64)
+        qs_p, nq = qs.ctypes.data_as(ctypes.c_void_p), qs.shape[0]
+    rc = lib().oracle_pcpp_attention_stale(qp, kp, vp, ksp, vsp, gkp, gvp, out.ctypes.data_as(ctypes.c_void_p),
+                                           B, heads, H, W, d, n_strips, float(p), G, qs_p, nq)
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return out
+
+
 # ---------------------------------------------------------------------------
 # Dense formulation: a membership predicate over coordinates, then a masked
 # softmax over the full key axis.
@@ -215,3 +244,35 @@ def dense_attention(q, k, v, *, geometry: str, B, heads, H, W, d, gk=None, gv=No
     w = np.exp(logits)
     w /= w.sum(axis=-1, keepdims=True)
     return np.einsum("bhtj,bhjc->bhtc", w, V)
+
+
+def dense_pcpp_stale(q, k, v, ks, vs, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None, G=0) -> np.ndarray:
+    """Dense form of the two-source PCPP: logits against the current keys where
+    the key row shares the query's strip and against the stale keys elsewhere,
+    one masked softmax over all keys, values picked the same way."""
+    N = H * W
+    mask = dense_mask("pcpp", H, W, n_strips=n_strips, p=p, G=G)
+    strip = (np.arange(N) // W) // (H // n_strips)
+    own = strip[:, None] == strip[None, :]                      # [N, N] same strip
+    Q = bf16_to_f64(q).reshape(B, heads, N, d)
+    Kf = bf16_to_f64(k).reshape(B, heads, N, d)
+    Vf = bf16_to_f64(v).reshape(B, heads, N, d)
+    Ks = bf16_to_f64(ks).reshape(B, heads, N, d)
+    Vs = bf16_to_f64(vs).reshape(B, heads, N, d)
+    lf = np.einsum("bhtc,bhjc->bhtj", Q, Kf)
+    ls = np.einsum("bhtc,bhjc->bhtj", Q, Ks)
+    logits = np.where(own[None, None], lf, ls)
+    if G:
+        lg = np.einsum("bhtc,bhjc->bhtj", Q, bf16_to_f64(gk).reshape(B, heads, G, d))
+        logits = np.concatenate([logits, lg], axis=-1)
+    logits = logits / np.sqrt(d)
+    logits = np.where(mask[None, None], logits, -np.inf)
+    logits -= logits.max(axis=-1, keepdims=True)
+    w = np.exp(logits)
+    w /= w.sum(axis=-1, keepdims=True)
+    wi = w[..., :N]
+    out = np.einsum("bhtj,bhjc->bhtc", np.where(own[None, None], wi, 0.0), Vf)
+    out += np.einsum("bhtj,bhjc->bhtc", np.where(own[None, None], 0.0, wi), Vs)
+    if G:
+        out += np.einsum("bhtj,bhjc->bhtc", w[..., N:], bf16_to_f64(gv).reshape(B, heads, G, d))
+    return out

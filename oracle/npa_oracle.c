@@ -133,15 +133,18 @@ int oracle_pcpp_key_set(int H, int W, int n_strips, double p, int t, int32_t *ou
 /* ------------------------------------------------------------------ */
 
 /* One query row. keys: n_img image token ids into k/v (rows of d), then all
- * G global rows. Scratch z must hold n_img + G doubles. */
+ * G global rows. When stale[j] is set, image key j is read from ks/vs instead
+ * of k/v. Scratch z must hold n_img + G doubles. */
 static int attend_one(const uint16_t *q_row, const uint16_t *k_bh, const uint16_t *v_bh,
+                      const uint16_t *ks_bh, const uint16_t *vs_bh, const unsigned char *stale,
                       const uint16_t *gk_bh, const uint16_t *gv_bh, int G, int d,
                       const int32_t *keys, int n_img, double *z, double *o_row) {
     const double scale = 1.0 / sqrt((double)d);
     int n = n_img + G;
     double m = -INFINITY;
     for (int j = 0; j < n; ++j) {
-        const uint16_t *kr = j < n_img ? k_bh + (size_t)keys[j] * d : gk_bh + (size_t)(j - n_img) * d;
+        const uint16_t *kr = j >= n_img ? gk_bh + (size_t)(j - n_img) * d
+                           : (stale && stale[j] ? ks_bh : k_bh) + (size_t)keys[j] * d;
         double dot = 0.0;
         for (int c = 0; c < d; ++c) dot += bf16_to_double(q_row[c]) * bf16_to_double(kr[c]);
         z[j] = dot * scale;
@@ -157,7 +160,8 @@ static int attend_one(const uint16_t *q_row, const uint16_t *k_bh, const uint16_
     for (int j = 0; j < n; ++j) {
         double w = z[j] / l;
         wsum += w;
-        const uint16_t *vr = j < n_img ? v_bh + (size_t)keys[j] * d : gv_bh + (size_t)(j - n_img) * d;
+        const uint16_t *vr = j >= n_img ? gv_bh + (size_t)(j - n_img) * d
+                           : (stale && stale[j] ? vs_bh : v_bh) + (size_t)keys[j] * d;
         for (int c = 0; c < d; ++c) o_row[c] += w * bf16_to_double(vr[c]);
     }
     if (fabs(wsum - 1.0) > 1e-12) return ORACLE_SUM_CHECK;
@@ -173,13 +177,16 @@ static int key_set(int geom, int H, int W, int a, int b, double p, int t, int32_
 /* Runs attention for a list of queries. queries holds n_queries triples
  * (b, h, t); out_rows receives n_queries rows of d doubles, in list order.
  * When queries is NULL, every (b, h, t) is computed and out_rows is the full
- * [B, heads, H*W, d] tensor. */
+ * [B, heads, H*W, d] tensor. For PCPP with ks/vs given, the keys of a query's
+ * own strip come from k/v and the neighbour rows from ks/vs. */
 static int run(int geom, const uint16_t *q, const uint16_t *k, const uint16_t *v,
+               const uint16_t *ks, const uint16_t *vs,
                const uint16_t *gk, const uint16_t *gv, double *out_rows,
                int B, int heads, int H, int W, int d, int a, int b, double p, int G,
                const int32_t *queries, long n_queries) {
     if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || G < 0) return ORACLE_BAD_ARG;
     if (G > 0 && (!gk || !gv)) return ORACLE_BAD_ARG;
+    if ((ks != NULL) != (vs != NULL) || (ks && geom != 1)) return ORACLE_BAD_ARG;
     const long N = (long)H * W;
     const long total = queries ? n_queries : (long)B * heads * N;
     int status = ORACLE_OK;
@@ -195,7 +202,8 @@ static int run(int geom, const uint16_t *q, const uint16_t *k, const uint16_t *v
     {
         int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
         double *z = (double *)malloc(sizeof(double) * (size_t)(N + G));
-        if (!keys || !z) {
+        unsigned char *stale = ks ? (unsigned char *)malloc((size_t)N) : NULL;
+        if (!keys || !z || (ks && !stale)) {
 #pragma omp critical
             status = ORACLE_NOMEM;
         } else {
@@ -217,8 +225,14 @@ static int run(int geom, const uint16_t *q, const uint16_t *k, const uint16_t *v
                 const uint16_t *gk_bh = G ? gk + bh * (size_t)G * d : NULL;
                 const uint16_t *gv_bh = G ? gv + bh * (size_t)G * d : NULL;
                 int n_img = key_set(geom, H, W, a, b, p, (int)t, keys);
-                int rc = attend_one(q + (bh * N + t) * d, k_bh, v_bh, gk_bh, gv_bh, G, d, keys, n_img, z,
-                                    out_rows + (size_t)i * d);
+                const uint16_t *ks_bh = ks ? ks + bh * N * d : NULL, *vs_bh = vs ? vs + bh * N * d : NULL;
+                if (stale) {
+                    /* a key is stale when its row lies outside the query's own strip */
+                    int s_rows = H / a, own = (int)(t / W) / s_rows;
+                    for (int j = 0; j < n_img; ++j) stale[j] = (unsigned char)((keys[j] / W) / s_rows != own);
+                }
+                int rc = attend_one(q + (bh * N + t) * d, k_bh, v_bh, ks_bh, vs_bh, stale, gk_bh, gv_bh, G, d, keys,
+                                    n_img, z, out_rows + (size_t)i * d);
                 if (rc != ORACLE_OK) {
 #pragma omp critical
                     status = rc;
@@ -227,6 +241,7 @@ static int run(int geom, const uint16_t *q, const uint16_t *k, const uint16_t *v
         }
         free(keys);
         free(z);
+        free(stale);
     }
     return status;
 }
@@ -235,14 +250,27 @@ int oracle_npa_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v
                          const uint16_t *gk, const uint16_t *gv, double *out,
                          int B, int heads, int H, int W, int d, int P, int m, int G,
                          const int32_t *queries, long n_queries) {
-    return run(0, q, k, v, gk, gv, out, B, heads, H, W, d, P, m, 0.0, G, queries, n_queries);
+    return run(0, q, k, v, NULL, NULL, gk, gv, out, B, heads, H, W, d, P, m, 0.0, G, queries, n_queries);
 }
 
 int oracle_pcpp_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                           const uint16_t *gk, const uint16_t *gv, double *out,
                           int B, int heads, int H, int W, int d, int n_strips, double p, int G,
                           const int32_t *queries, long n_queries) {
-    return run(1, q, k, v, gk, gv, out, B, heads, H, W, d, n_strips, 0, p, G, queries, n_queries);
+    return run(1, q, k, v, NULL, NULL, gk, gv, out, B, heads, H, W, d, n_strips, 0, p, G, queries, n_queries);
+}
+
+/* PCPP with stale neighbour rows (PCPP review, "Core claim": a patch is
+ * updated from its own activation plus the top or bottom p-fraction of the
+ * neighbouring patches *from the previous step*): keys of the query's own
+ * strip from k/v, the neighbour rows from ks/vs (same layout). */
+int oracle_pcpp_attention_stale(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                const uint16_t *ks, const uint16_t *vs,
+                                const uint16_t *gk, const uint16_t *gv, double *out,
+                                int B, int heads, int H, int W, int d, int n_strips, double p, int G,
+                                const int32_t *queries, long n_queries) {
+    if (!ks || !vs) return ORACLE_BAD_ARG;
+    return run(1, q, k, v, ks, vs, gk, gv, out, B, heads, H, W, d, n_strips, 0, p, G, queries, n_queries);
 }
 
 /* Number of (query, key) pairs, summed over all queries of one (b, h),
