@@ -94,6 +94,23 @@ npa_status pcpp_attention_fwd(const void *q, const void *k, const void *v, void 
                               int B, int heads, int H, int W, int d, int n_strips, double p,
                               const npa_global_kv *global_kv, npa_stream_t stream);
 
+/* Partially conditioned attention with stale neighbour rows, the form PCPP
+ * runs across devices (PCPP review, "Core claim": a patch is updated from its
+ * own activation plus the top or bottom p-fraction of the neighbouring
+ * patches from the previous denoising step). For the queries of strips
+ * [strip_begin, strip_begin + strip_count) the keys/values of the query's own
+ * strip are read from k, v (current step) and the borrowed neighbour rows
+ * from k_stale, v_stale (previous step; same layout and size as k, v; only
+ * the r rows next to each computed strip are read). Output rows of other
+ * strips are left untouched. Other arguments and errors as for
+ * pcpp_attention_fwd; 0 <= strip_begin, 1 <= strip_count,
+ * strip_begin + strip_count <= n_strips, and o must not overlap k_stale or
+ * v_stale. */
+npa_status pcpp_attention_fwd_stale(const void *q, const void *k, const void *v, const void *k_stale,
+                                    const void *v_stale, void *o, int B, int heads, int H, int W, int d,
+                                    int n_strips, double p, int strip_begin, int strip_count,
+                                    const npa_global_kv *global_kv, npa_stream_t stream);
+
 /* r = ceil(p * strip_rows) (double, 1e-9 allowance), limited to
  * [0, strip_rows]. Returns -1 if strip_rows < 1 or p is outside [0, 1]. */
 int pcpp_neighbor_rows(int strip_rows, double p);

@@ -24,7 +24,7 @@ __all__ = [
     "NPA_ERR_MISALIGNED", "NPA_ERR_CUDA", "NPA_ERR_DEVICE_TIMEOUT", "npa_attention_fwd",
     "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops", "pcpp_useful_flops",
     "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string", "npa_attention",
-    "pcpp_attention", "EXPORTED_SYMBOLS",
+    "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
@@ -37,7 +37,7 @@ NPA_ERR_CUDA = 4
 NPA_ERR_DEVICE_TIMEOUT = 5
 
 EXPORTED_SYMBOLS = (
-    "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops",
+    "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_attention_fwd_stale", "pcpp_neighbor_rows", "npa_useful_flops",
     "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
 )
 
@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.npa_attention_fwd.restype = i
         L.pcpp_attention_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, d, gkv, vp]
         L.pcpp_attention_fwd.restype = i
+        L.pcpp_attention_fwd_stale.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, d, i, i, gkv, vp]
+        L.pcpp_attention_fwd_stale.restype = i
         L.pcpp_neighbor_rows.argtypes = [i, d]
         L.pcpp_neighbor_rows.restype = i
         L.npa_useful_flops.argtypes = [i, i, i, i, i, i, i, i]
@@ -134,6 +136,16 @@ def pcpp_attention_fwd(q, k, v, o, B: int, heads: int, H: int, W: int, d: int, n
            "pcpp_attention_fwd")
 
 
+def pcpp_attention_fwd_stale(q, k, v, k_stale, v_stale, o, B: int, heads: int, H: int, W: int, d: int,
+                             n_strips: int, p: float, strip_begin: int, strip_count: int, global_k=None,
+                             global_v=None, n_global: int = 0, stream=None) -> None:
+    """C ``pcpp_attention_fwd_stale``: own-strip keys from k/v, borrowed rows from k_stale/v_stale."""
+    _check(lib().pcpp_attention_fwd_stale(_ptr(q), _ptr(k), _ptr(v), _ptr(k_stale), _ptr(v_stale), _ptr(o), B,
+                                          heads, H, W, d, n_strips, float(p), strip_begin, strip_count,
+                                          _gkv(global_k, global_v, n_global), _stream(stream)),
+           "pcpp_attention_fwd_stale")
+
+
 def pcpp_neighbor_rows(strip_rows: int, p: float) -> int:
     return int(lib().pcpp_neighbor_rows(strip_rows, float(p)))
 
@@ -190,4 +202,18 @@ def pcpp_attention(q, k, v, H: int, W: int, n_strips: int, p: float, global_k=No
         out = q.new_empty(q.shape)
     G = 0 if global_k is None else int(global_k.shape[2])
     pcpp_attention_fwd(q, k, v, out, B, heads, H, W, d, n_strips, p, global_k, global_v, G, stream)
+    return out
+
+
+def pcpp_attention_stale(q, k, v, k_stale, v_stale, H: int, W: int, n_strips: int, p: float, strips=None,
+                         global_k=None, global_v=None, out=None, stream=None):
+    """Two-source PCPP forward on torch bf16 CUDA tensors; ``strips`` is an
+    optional (begin, count) range of strips to compute (default: all)."""
+    B, heads, d = _shape(q, H, W)
+    if out is None:
+        out = q.new_empty(q.shape)
+    begin, count = (0, n_strips) if strips is None else strips
+    G = 0 if global_k is None else int(global_k.shape[2])
+    pcpp_attention_fwd_stale(q, k, v, k_stale, v_stale, out, B, heads, H, W, d, n_strips, p, begin, count,
+                             global_k, global_v, G, stream)
     return out

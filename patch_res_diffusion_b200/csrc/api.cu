@@ -191,38 +191,44 @@ npa_status validate_common(const void *q, const void *k, const void *v, void *o,
 // Patches ordered by decreasing number of key blocks (ties: natural order),
 // so a persistent CTA's last units are its cheapest.
 void order_patches(const Geo &g, FwdParams &prm) {
-    const int np = prm.nPh * prm.nPw;
+    const int np = prm.patch_count;
     if (np > npa::kMaxPatchOrder) {
         prm.n_perm = 0;
         return;
     }
     const int kc = 1 << prm.kc_log2;
-    int cost[npa::kMaxPatchOrder];
-    for (int pi = 0; pi < prm.nPh; ++pi) {
-        for (int pj = 0; pj < prm.nPw; ++pj) {
-            const int r0 = pi * g.Ph, r1 = r0 + g.Ph < g.H ? r0 + g.Ph : g.H;
-            const int c0 = pj * g.Pw, c1 = c0 + g.Pw < g.W ? c0 + g.Pw : g.W;
-            const int wh = (r1 + g.mh < g.H ? r1 + g.mh : g.H) - (r0 - g.mh > 0 ? r0 - g.mh : 0);
-            const int ww = (c1 + g.mw < g.W ? c1 + g.mw : g.W) - (c0 - g.mw > 0 ? c0 - g.mw : 0);
-            cost[pi * prm.nPw + pj] = ((ww + kc - 1) / kc) * ((wh + prm.kr - 1) / prm.kr);
-        }
+    int cost[npa::kMaxPatchOrder];  // indexed by position in the patch range
+    for (int i = 0; i < np; ++i) {
+        const int patch = prm.patch_begin + i;
+        const int pi = patch / prm.nPw, pj = patch % prm.nPw;
+        const int r0 = pi * g.Ph, r1 = r0 + g.Ph < g.H ? r0 + g.Ph : g.H;
+        const int c0 = pj * g.Pw, c1 = c0 + g.Pw < g.W ? c0 + g.Pw : g.W;
+        const int wh = (r1 + g.mh < g.H ? r1 + g.mh : g.H) - (r0 - g.mh > 0 ? r0 - g.mh : 0);
+        const int ww = (c1 + g.mw < g.W ? c1 + g.mw : g.W) - (c0 - g.mw > 0 ? c0 - g.mw : 0);
+        cost[i] = ((ww + kc - 1) / kc) * ((wh + prm.kr - 1) / prm.kr);
     }
-    for (int i = 0; i < np; ++i) prm.patch_order[i] = (unsigned short)i;
+    unsigned short idx[npa::kMaxPatchOrder];
+    for (int i = 0; i < np; ++i) idx[i] = (unsigned short)i;
     // insertion sort, stable, descending cost (np <= 256)
     for (int i = 1; i < np; ++i) {
-        const unsigned short x = prm.patch_order[i];
+        const unsigned short x = idx[i];
         int j = i - 1;
-        while (j >= 0 && cost[prm.patch_order[j]] < cost[x]) {
-            prm.patch_order[j + 1] = prm.patch_order[j];
+        while (j >= 0 && cost[idx[j]] < cost[x]) {
+            idx[j + 1] = idx[j];
             --j;
         }
-        prm.patch_order[j + 1] = x;
+        idx[j + 1] = x;
     }
+    for (int i = 0; i < np; ++i) prm.patch_order[i] = (unsigned short)(prm.patch_begin + idx[i]);
     prm.n_perm = np;
 }
 
-npa_status launch(const void *q, const void *k, const void *v, void *o, int B, int heads, int d, const Geo &g,
-                  int G, const npa_global_kv *gkv, npa_stream_t stream) {
+// ks / vs (both or neither): previous-step keys/values for the rows of a
+// window outside its patch. [patch_begin, patch_begin + patch_count): the
+// patches computed, in natural numbering; patch_count < 0 means all.
+npa_status launch(const void *q, const void *k, const void *v, const void *ks, const void *vs, void *o, int B,
+                  int heads, int d, const Geo &g, int G, const npa_global_kv *gkv, int patch_begin, int patch_count,
+                  npa_stream_t stream) {
     int sm_count = 0;
     npa_status st = ensure_ready(&sm_count);
     if (st != NPA_OK) return st;
@@ -248,8 +254,12 @@ npa_status launch(const void *q, const void *k, const void *v, void *o, int B, i
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     prm.wait_limit_ns = kWaitLimitNs;
 
-    const long long units = (long long)B * heads * prm.nPh * prm.nPw * prm.n_qblocks;
-    if (units > INT_MAX / 2 || (long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
+    if ((long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
+    prm.patch_begin = patch_begin;
+    prm.patch_count = patch_count < 0 ? prm.nPh * prm.nPw : patch_count;
+    prm.two_source = ks != nullptr;
+    const long long units = (long long)B * heads * prm.patch_count * prm.n_qblocks;
+    if (units > INT_MAX / 2) return NPA_ERR_UNSUPPORTED;
 
     const int BH = B * heads;
     prm.BH = BH;
@@ -264,6 +274,8 @@ npa_status launch(const void *q, const void *k, const void *v, void *o, int B, i
     const cuuint32_t kbox[4] = {64, (cuuint32_t)(1 << prm.kc_log2), (cuuint32_t)prm.kr, 1};
     if (!encode(&prm.tm_q, q, 4, dims, strides, qbox) || !encode(&prm.tm_k, k, 4, dims, strides, kbox) ||
         !encode(&prm.tm_v, v, 4, dims, strides, kbox))
+        return NPA_ERR_CUDA;
+    if (ks && (!encode(&prm.tm_ks, ks, 4, dims, strides, kbox) || !encode(&prm.tm_vs, vs, 4, dims, strides, kbox)))
         return NPA_ERR_CUDA;
     if (G > 0) {
         const cuuint64_t gdims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)BH};
@@ -310,7 +322,7 @@ npa_status npa_attention_fwd(const void *q, const void *k, const void *v, void *
     if (st != NPA_OK) return st;
     if (patch < 1 || margin < 0) return NPA_ERR_INVALID_ARG;
     const Geo g{H, W, patch, patch, margin, margin};
-    return launch(q, k, v, o, B, heads, d, g, G, global_kv, stream);
+    return launch(q, k, v, nullptr, nullptr, o, B, heads, d, g, G, global_kv, 0, -1, stream);
 }
 
 npa_status pcpp_attention_fwd(const void *q, const void *k, const void *v, void *o, int B, int heads, int H, int W,
@@ -321,7 +333,25 @@ npa_status pcpp_attention_fwd(const void *q, const void *k, const void *v, void 
     if (n_strips < 1 || H % n_strips != 0 || !(p >= 0.0) || !(p <= 1.0)) return NPA_ERR_INVALID_ARG;
     const int s = H / n_strips;
     const Geo g{H, W, s, W, neighbor_rows(s, p), 0};
-    return launch(q, k, v, o, B, heads, d, g, G, global_kv, stream);
+    return launch(q, k, v, nullptr, nullptr, o, B, heads, d, g, G, global_kv, 0, -1, stream);
+}
+
+npa_status pcpp_attention_fwd_stale(const void *q, const void *k, const void *v, const void *k_stale,
+                                    const void *v_stale, void *o, int B, int heads, int H, int W, int d, int n_strips,
+                                    double p, int strip_begin, int strip_count, const npa_global_kv *global_kv,
+                                    npa_stream_t stream) {
+    int G = 0;
+    npa_status st = validate_common(q, k, v, o, B, heads, H, W, d, global_kv, &G);
+    if (st != NPA_OK) return st;
+    if (!k_stale || !v_stale) return NPA_ERR_INVALID_ARG;
+    if (!aligned16(k_stale) || !aligned16(v_stale)) return NPA_ERR_MISALIGNED;
+    const size_t bytes = (size_t)B * heads * H * W * d * 2;
+    if (overlaps(o, bytes, k_stale, bytes) || overlaps(o, bytes, v_stale, bytes)) return NPA_ERR_INVALID_ARG;
+    if (n_strips < 1 || H % n_strips != 0 || !(p >= 0.0) || !(p <= 1.0)) return NPA_ERR_INVALID_ARG;
+    if (strip_begin < 0 || strip_count < 1 || strip_begin > n_strips - strip_count) return NPA_ERR_INVALID_ARG;
+    const int s = H / n_strips;
+    const Geo g{H, W, s, W, neighbor_rows(s, p), 0};
+    return launch(q, k, v, k_stale, v_stale, o, B, heads, d, g, G, global_kv, strip_begin, strip_count, stream);
 }
 
 int pcpp_neighbor_rows(int strip_rows, double p) { return neighbor_rows(strip_rows, p); }

@@ -127,12 +127,11 @@ __device__ __forceinline__ void load_block(const FwdParams &p, const Work &w, in
                                            uint64_t *bar) {
     using C = KCfg<D>;
     if (j < w.n_win) {
-        const int tr = j / w.wtc, tc = j - tr * w.wtc;
-        const int col = w.wc0 + (tc << p.kc_log2), row = w.wr0 + tr * p.kr;
-        const CUtensorMap *m = is_v ? &p.tm_v : &p.tm_k;
+        const BlockGeom b = block_geom(p, w, j);
+        const CUtensorMap *m = b.stale ? (is_v ? &p.tm_vs : &p.tm_ks) : (is_v ? &p.tm_v : &p.tm_k);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_4d(dst + c * C::kChunkBytes, m, bar, c * 64, col, row, w.bh);
+            sm100::tma_load_4d(dst + c * C::kChunkBytes, m, bar, c * 64, b.col, b.row, w.bh);
     } else {
         const int g0 = (j - w.n_win) * 128;
         const CUtensorMap *m = is_v ? &p.tm_gv : &p.tm_gk;
@@ -152,6 +151,10 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
     if (p.G > 0) {
         sm100::tma_prefetch_desc(&p.tm_gk);
         sm100::tma_prefetch_desc(&p.tm_gv);
+    }
+    if (p.two_source) {
+        sm100::tma_prefetch_desc(&p.tm_ks);
+        sm100::tma_prefetch_desc(&p.tm_vs);
     }
     const uint32_t q_bytes = uint32_t(C::kChunks * p.qc * p.qr * 128);
     int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q pairs issued
@@ -499,11 +502,15 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
     const Work w = decode_work(p, unit);
     if (!unit_has_work(p, w)) continue;
+    const int n_blocks = w.n_blocks;
+    // window block coordinates, advanced without divisions: column block,
+    // first row of the current band, end of the band's row segment
+    int btc = 0, brow = w.seg[0], bend = w.seg[1];
+    if (brow >= bend) bend = w.seg[2];
     float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
     float R_prev = -INFINITY;  // reference that O and l are currently expressed in
     float l = 0.f;
-    int btc = 0, btr = 0;      // window block coordinates of block j
-    for (int j = 0; j < w.n_blocks; ++j, ++gb) {
+    for (int j = 0; j < n_blocks; ++j, ++gb) {
         if (!warp_wait(&bars[C::bSFull + q], gb & 1, lim)) {
             ok = false;
             break;
@@ -521,10 +528,11 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             sm100::tc_fence_before();
             sm100::mbar_arrive(&bars[C::bSFree + q]);
         }
-        // keys of this block outside the window (or past the last global token) get -inf
+        // keys of this block outside its row segment or the window (or past
+        // the last global token) get -inf
         if (j < w.n_win) {
             const int vc = w.wc1 - (w.wc0 + (btc << p.kc_log2));
-            const int vr = w.wr1 - (w.wr0 + btr * p.kr);
+            const int vr = bend - brow;
             if (vc < kc || vr < p.kr) {
 #pragma unroll
                 for (int i = 0; i < 128; ++i)
@@ -532,7 +540,11 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
             if (++btc == w.wtc) {
                 btc = 0;
-                ++btr;
+                brow += p.kr;
+                if (brow >= bend) {  // next row segment
+                    brow = bend;
+                    bend = bend == w.seg[1] ? w.seg[2] : w.seg[3];
+                }
             }
         } else {
             const int vg = p.G - (j - w.n_win) * 128;

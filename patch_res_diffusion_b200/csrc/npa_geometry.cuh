@@ -33,6 +33,8 @@ struct FwdParams {
     CUtensorMap tm_v;   // 4D, box {64, kc, kr, 1}
     CUtensorMap tm_gk;  // 3D {d, G, B*heads}, box {64, 128, 1} (unused when G == 0)
     CUtensorMap tm_gv;
+    CUtensorMap tm_ks;  // previous step's K / V for the borrowed rows (two_source only)
+    CUtensorMap tm_vs;
     void *o;            // bf16 [B, heads, H*W, d]
     int H, W, G;
     int Ph, Pw, mh, mw;
@@ -44,17 +46,33 @@ struct FwdParams {
     unsigned long long wait_limit_ns;
     int BH;                          // batch * heads
     int n_units;                     // work units in execution order
+    int two_source;                  // 1: rows outside the patch come from tm_ks / tm_vs
+    int patch_begin, patch_count;    // patches computed (natural order when n_perm == 0)
     int n_perm;                      // entries of patch_order (0: natural order)
     unsigned short patch_order[kMaxPatchOrder];  // patches by decreasing window area
 };
 
+// The window's rows are walked as three segments: [seg[0], seg[1]) and
+// [seg[2], seg[3]) are read from the previous step's keys/values (two-source
+// PCPP: the borrowed neighbour rows) and [seg[1], seg[2]) from the current
+// ones. With one source the outer segments are empty.
 struct Work {
     int bh;
     int pr0, pr1, pc0, pc1;   // clipped patch
     int wr0, wr1, wc0, wc1;   // clipped window
+    int seg[4];               // row segment boundaries (see above)
+    int nb0, nb01;            // key blocks of segment 0, of segments 0 and 1
     int tile0;                // first query tile (of two) within the patch
     int wtc;                  // window blocks along the columns
     int n_win, n_blocks;      // window blocks, window + global blocks
+};
+
+// Where key block j (< n_win) of a unit lies: first row and column of its box,
+// how many of its rows and columns are inside its segment and the window, and
+// whether it is read from the previous step's buffers.
+struct BlockGeom {
+    int row, col, vr, vc;
+    bool stale;
 };
 
 __host__ __device__ inline int imin_(int a, int b) { return a < b ? a : b; }
@@ -70,7 +88,7 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     const int rest = unit / p.n_qblocks;
     w.bh = rest % p.BH;
     const int rank = rest / p.BH;
-    const int patch = rank < p.n_perm ? int(p.patch_order[rank]) : rank;
+    const int patch = p.n_perm ? int(p.patch_order[rank]) : p.patch_begin + rank;
     const int pi = patch / p.nPw, pj = patch % p.nPw;
     w.pr0 = pi * p.Ph;
     w.pr1 = imin_(p.H, w.pr0 + p.Ph);
@@ -83,9 +101,36 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     w.tile0 = 2 * qb;
     const int kc = 1 << p.kc_log2;
     w.wtc = cdiv_(w.wc1 - w.wc0, kc);
-    w.n_win = w.wtc * cdiv_(w.wr1 - w.wr0, p.kr);
+    if (p.two_source) {
+        w.seg[0] = w.wr0;
+        w.seg[1] = w.pr0;
+        w.seg[2] = w.pr1;
+        w.seg[3] = w.wr1;
+    } else {
+        w.seg[0] = w.seg[1] = w.wr0;
+        w.seg[2] = w.seg[3] = w.wr1;
+    }
+    w.nb0 = w.wtc * cdiv_(w.seg[1] - w.seg[0], p.kr);
+    w.nb01 = w.nb0 + w.wtc * cdiv_(w.seg[2] - w.seg[1], p.kr);
+    w.n_win = w.nb01 + w.wtc * cdiv_(w.seg[3] - w.seg[2], p.kr);
     w.n_blocks = w.n_win + cdiv_(p.G, 128);
     return w;
+}
+
+__host__ __device__ inline BlockGeom block_geom(const FwdParams &p, const Work &w, int j) {
+    const int sg = j < w.nb0 ? 0 : (j < w.nb01 ? 1 : 2);
+    const int l = j - (sg == 0 ? 0 : (sg == 1 ? w.nb0 : w.nb01));
+    const int tr = l / w.wtc, tc = l - tr * w.wtc;
+    // selects, not a runtime index, so the segment bounds stay in registers
+    const int lo = sg == 0 ? w.seg[0] : (sg == 1 ? w.seg[1] : w.seg[2]);
+    const int hi = sg == 0 ? w.seg[1] : (sg == 1 ? w.seg[2] : w.seg[3]);
+    BlockGeom b;
+    b.row = lo + tr * p.kr;
+    b.col = w.wc0 + (tc << p.kc_log2);
+    b.vr = imin_(p.kr, hi - b.row);
+    b.vc = imin_(1 << p.kc_log2, w.wc1 - b.col);
+    b.stale = sg != 1;
+    return b;
 }
 
 // Origin (first row, first column) of query tile t of the unit's patch.

@@ -142,3 +142,20 @@ def test_flops_helper_rejects_bad_geometry():
     assert npa.npa_useful_flops(1, 1, 8, 8, 64, 0, 1) < 0
     assert npa.pcpp_useful_flops(1, 1, 9, 8, 64, 2, 0.5) < 0
     assert npa.pcpp_useful_flops(1, 1, 8, 8, 64, 2, 1.5) < 0
+
+
+def _stale(L, q=A, k=B_, v=C_, ks=0x30000000, vs=0x50000000, o=O_, H=8, n=2, p=0.5, b=0, c=1, d=64):
+    return L.pcpp_attention_fwd_stale(q, k, v, ks, vs, o, 1, 1, H, 8, d, n, p, b, c, None, None)
+
+
+def test_stale_entry_point_validation(L):
+    assert _stale(L, ks=None) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, vs=None) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, ks=0x30000008) == npa.NPA_ERR_MISALIGNED
+    assert _stale(L, o=0x30000000) == npa.NPA_ERR_INVALID_ARG       # output overlaps k_stale
+    assert _stale(L, b=-1) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, c=0) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, b=1, c=2) == npa.NPA_ERR_INVALID_ARG            # past the last strip
+    assert _stale(L, H=9) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, p=2.0) == npa.NPA_ERR_INVALID_ARG
+    assert _stale(L, d=96) == npa.NPA_ERR_UNSUPPORTED
