@@ -148,7 +148,7 @@ def run_reference(args, w: Workload, rank: int) -> None:
         return
     inp = make_inputs(w)
     steps = []
-    budget = max(1.0, 30.0 / max(1, args.steps + args.warmup))
+    budget = max(0.5, min(2.0 * args.cpu_seconds, 30.0) / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         r = oracle_rate(w, inp, budget)
         if i >= args.warmup:
