@@ -35,7 +35,7 @@ from . import build as _build
 __all__ = [
     "lib", "npa_key_set", "pcpp_key_set", "pcpp_neighbor_rows", "npa_attention",
     "pcpp_attention", "pcpp_attention_stale", "pair_count", "num_threads", "dense_mask",
-    "dense_attention", "dense_pcpp_stale", "bf16_to_f64",
+    "dense_attention", "dense_pcpp_stale", "global_query_attention", "bf16_to_f64",
 ]
 
 _LIB = None
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         L.oracle_pcpp_attention_stale.argtypes = [u16p] * 7 + [ctypes.c_void_p] + [ctypes.c_int] * 5 + [
             ctypes.c_int, ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_long]
         L.oracle_pcpp_attention_stale.restype = ctypes.c_int
+        L.oracle_global_query_attention.argtypes = [u16p] * 5 + [ctypes.c_void_p] + [ctypes.c_int] * 6 + [
+            ctypes.c_void_p, ctypes.c_long]
+        L.oracle_global_query_attention.restype = ctypes.c_int
         L.oracle_pair_count.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
         L.oracle_pair_count.restype = ctypes.c_longlong
         L.oracle_num_threads.argtypes = []
@@ -177,6 +180,30 @@ def pcpp_attention_stale(q, k, v, ks, vs, *, B, heads, H, W, d, n_strips, p, gk=
         qs_p, nq = qs.ctypes.data_as(ctypes.c_void_p), qs.shape[0]
     rc = lib().oracle_pcpp_attention_stale(qp, kp, vp, ksp, vsp, gkp, gvp, out.ctypes.data_as(ctypes.c_void_p),
                                            B, heads, H, W, d, n_strips, float(p), G, qs_p, nq)
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return out
+
+
+def global_query_attention(gq, k, v, gk, gv, *, B, heads, H, W, d, G,
+                           queries: Optional[Sequence] = None) -> np.ndarray:
+    """Text-query half of joint attention, float64: each global token attends
+    to all H*W image tokens and all G global tokens. ``queries``: optional
+    (n, 3) array of (b, h, g); otherwise the full [B, heads, G, d] result."""
+    gq, gqp = _u16(gq)
+    k, kp = _u16(k)
+    v, vp = _u16(v)
+    gk, gkp = _u16(gk)
+    gv, gvp = _u16(gv)
+    if queries is None:
+        out = np.empty((B, heads, G, d), dtype=np.float64)
+        qs_p, nq = None, 0
+    else:
+        qs = np.ascontiguousarray(np.asarray(queries, dtype=np.int32).reshape(-1, 3))
+        out = np.empty((qs.shape[0], d), dtype=np.float64)
+        qs_p, nq = qs.ctypes.data_as(ctypes.c_void_p), qs.shape[0]
+    rc = lib().oracle_global_query_attention(gqp, kp, vp, gkp, gvp, out.ctypes.data_as(ctypes.c_void_p), B, heads,
+                                             H, W, d, G, qs_p, nq)
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
     return out

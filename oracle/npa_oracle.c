@@ -273,6 +273,58 @@ int oracle_pcpp_attention_stale(const uint16_t *q, const uint16_t *k, const uint
     return run(1, q, k, v, ks, vs, gk, gv, out, B, heads, H, W, d, n_strips, 0, p, G, queries, n_queries);
 }
 
+/* Text-query half of joint attention: the G global tokens as queries, each
+ * attending to every image token and every global token (full attention;
+ * the pages leave the text tokens unrestricted - ScaleDiff summary: NPA
+ * restricts the image-token queries of self-attention). gq, out: [B, heads,
+ * G, d]; queries: optional (b, h, g) triples. */
+int oracle_global_query_attention(const uint16_t *gq, const uint16_t *k, const uint16_t *v,
+                                  const uint16_t *gk, const uint16_t *gv, double *out,
+                                  int B, int heads, int H, int W, int d, int G,
+                                  const int32_t *queries, long n_queries) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || G < 1 || !gq || !k || !v || !gk || !gv)
+        return ORACLE_BAD_ARG;
+    const long N = (long)H * W;
+    const long total = queries ? n_queries : (long)B * heads * G;
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+        double *z = (double *)malloc(sizeof(double) * (size_t)(N + G));
+        if (!keys || !z) {
+#pragma omp critical
+            status = ORACLE_NOMEM;
+        } else {
+            for (long j = 0; j < N; ++j) keys[j] = (int32_t)j;   /* every image token */
+#pragma omp for schedule(dynamic, 16)
+            for (long i = 0; i < total; ++i) {
+                long bb, hh, g;
+                if (queries) {
+                    bb = queries[3 * i]; hh = queries[3 * i + 1]; g = queries[3 * i + 2];
+                    if (bb < 0 || bb >= B || hh < 0 || hh >= heads || g < 0 || g >= G) {
+#pragma omp critical
+                        status = ORACLE_BAD_ARG;
+                        continue;
+                    }
+                } else {
+                    g = i % G; hh = (i / G) % heads; bb = i / ((long)G * heads);
+                }
+                size_t bh = (size_t)bb * heads + hh;
+                int rc = attend_one(gq + (bh * G + g) * d, k + bh * N * d, v + bh * N * d, NULL, NULL, NULL,
+                                    gk + bh * (size_t)G * d, gv + bh * (size_t)G * d, G, d, keys, (int)N, z,
+                                    out + (size_t)i * d);
+                if (rc != ORACLE_OK) {
+#pragma omp critical
+                    status = rc;
+                }
+            }
+        }
+        free(keys);
+        free(z);
+    }
+    return status;
+}
+
 /* Number of (query, key) pairs, summed over all queries of one (b, h),
  * counting image keys and global keys. Brute force over every token. */
 long long oracle_pair_count(int geom, int H, int W, int a, int b, double p, int G) {
