@@ -52,6 +52,7 @@
 #ifndef NPA_B200_H
 #define NPA_B200_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -110,6 +111,28 @@ npa_status pcpp_attention_fwd_stale(const void *q, const void *k, const void *v,
                                     const void *v_stale, void *o, int B, int heads, int H, int W, int d,
                                     int n_strips, double p, int strip_begin, int strip_count,
                                     const npa_global_kv *global_kv, npa_stream_t stream);
+
+/* Text-query half of joint (MM-DiT) attention: the G global tokens as
+ * queries, each attending to all H*W image tokens and all G global tokens
+ * (full attention). The pages restrict only the image-token queries
+ * (ScaleDiff summary, "Approach": NPA replaces the image self-attention; it
+ * extends to FLUX, whose text tokens join that attention), so the text
+ * queries are left unrestricted here.
+ * gq, go: bfloat16 [B, heads, G, d]; k, v: [B, heads, H*W, d]; gk, gv:
+ * [B, heads, G, d] (device). The key range is split across CTAs when the
+ * query tiles alone would leave most of the GPU idle; the partial results go
+ * to `workspace` (caller-owned device memory, 16-byte aligned, at least
+ * npa_global_query_workspace_size() bytes for the full split count; a
+ * smaller or NULL workspace gives fewer or no splits - same result, less
+ * parallelism) and are merged by a second kernel on the same stream. go must
+ * not overlap the inputs or the workspace. */
+npa_status npa_global_query_attention_fwd(const void *gq, const void *k, const void *v, const void *gk,
+                                          const void *gv, void *go, int B, int heads, int H, int W, int d,
+                                          int G, void *workspace, size_t workspace_bytes, npa_stream_t stream);
+
+/* Workspace bytes npa_global_query_attention_fwd uses for its full split
+ * count on the current device (0: no split needed, or invalid arguments). */
+size_t npa_global_query_workspace_size(int B, int heads, int H, int W, int d, int G);
 
 /* r = ceil(p * strip_rows) (double, 1e-9 allowance), limited to
  * [0, strip_rows]. Returns -1 if strip_rows < 1 or p is outside [0, 1]. */

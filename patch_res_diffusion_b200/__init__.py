@@ -24,7 +24,8 @@ __all__ = [
     "NPA_ERR_MISALIGNED", "NPA_ERR_CUDA", "NPA_ERR_DEVICE_TIMEOUT", "npa_attention_fwd",
     "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops", "pcpp_useful_flops",
     "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string", "npa_attention",
-    "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "EXPORTED_SYMBOLS",
+    "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "npa_global_query_attention_fwd",
+    "npa_global_query_workspace_size", "global_query_attention", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
@@ -39,6 +40,7 @@ NPA_ERR_DEVICE_TIMEOUT = 5
 EXPORTED_SYMBOLS = (
     "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_attention_fwd_stale", "pcpp_neighbor_rows", "npa_useful_flops",
     "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
+    "npa_global_query_attention_fwd", "npa_global_query_workspace_size",
 )
 
 
@@ -70,6 +72,10 @@ def lib() -> ctypes.CDLL:
         L.pcpp_attention_fwd.restype = i
         L.pcpp_attention_fwd_stale.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, d, i, i, gkv, vp]
         L.pcpp_attention_fwd_stale.restype = i
+        L.npa_global_query_attention_fwd.argtypes = [vp] * 6 + [i] * 6 + [vp, ctypes.c_size_t, vp]
+        L.npa_global_query_attention_fwd.restype = i
+        L.npa_global_query_workspace_size.argtypes = [i] * 6
+        L.npa_global_query_workspace_size.restype = ctypes.c_size_t
         L.pcpp_neighbor_rows.argtypes = [i, d]
         L.pcpp_neighbor_rows.restype = i
         L.npa_useful_flops.argtypes = [i, i, i, i, i, i, i, i]
@@ -146,6 +152,19 @@ def pcpp_attention_fwd_stale(q, k, v, k_stale, v_stale, o, B: int, heads: int, H
            "pcpp_attention_fwd_stale")
 
 
+def npa_global_query_attention_fwd(gq, k, v, gk, gv, go, B: int, heads: int, H: int, W: int, d: int, G: int,
+                                   workspace=None, workspace_bytes: int = 0, stream=None) -> None:
+    """C ``npa_global_query_attention_fwd``: global-token queries over all keys."""
+    _check(lib().npa_global_query_attention_fwd(_ptr(gq), _ptr(k), _ptr(v), _ptr(gk), _ptr(gv), _ptr(go), B, heads,
+                                                H, W, d, G, _ptr(workspace), int(workspace_bytes),
+                                                _stream(stream)),
+           "npa_global_query_attention_fwd")
+
+
+def npa_global_query_workspace_size(B, heads, H, W, d, G) -> int:
+    return int(lib().npa_global_query_workspace_size(B, heads, H, W, d, G))
+
+
 def pcpp_neighbor_rows(strip_rows: int, p: float) -> int:
     return int(lib().pcpp_neighbor_rows(strip_rows, float(p)))
 
@@ -216,4 +235,21 @@ def pcpp_attention_stale(q, k, v, k_stale, v_stale, H: int, W: int, n_strips: in
     G = 0 if global_k is None else int(global_k.shape[2])
     pcpp_attention_fwd_stale(q, k, v, k_stale, v_stale, out, B, heads, H, W, d, n_strips, p, begin, count,
                              global_k, global_v, G, stream)
+    return out
+
+
+def global_query_attention(gq, k, v, gk, gv, H: int, W: int, out=None, split: bool = True, stream=None):
+    """Global-token queries [B, heads, G, d] over all image and global keys
+    (torch bf16 CUDA tensors); with ``split`` a workspace is allocated so the
+    key range can be split across the GPU."""
+    import torch
+    B, heads, G, d = (int(x) for x in gq.shape)
+    if out is None:
+        out = gq.new_empty(gq.shape)
+    ws, nbytes = None, 0
+    if split:
+        nbytes = npa_global_query_workspace_size(B, heads, H, W, d, G)
+        if nbytes:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=gq.device)
+    npa_global_query_attention_fwd(gq, k, v, gk, gv, out, B, heads, H, W, d, G, ws, nbytes, stream)
     return out

@@ -62,9 +62,14 @@ npa_status ensure_ready(int *sm_count = nullptr) {
             return NPA_ERR_CUDA;
         if (major != 10 || minor != 0) {
             ds.status = NPA_ERR_UNSUPPORTED;
-        } else if (cudaFuncSetAttribute(npa::npa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        } else if (cudaFuncSetAttribute(npa::npa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         npa::KCfg<64>::kSmemBytes) != cudaSuccess ||
-                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128, false>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        npa::KCfg<128>::kSmemBytes) != cudaSuccess ||
+                   cudaFuncSetAttribute(npa::npa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        npa::KCfg<64>::kSmemBytes) != cudaSuccess ||
+                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         npa::KCfg<128>::kSmemBytes) != cudaSuccess) {
             return NPA_ERR_CUDA;
         } else {
@@ -289,12 +294,121 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     void *args[1] = {&prm};
     cudaError_t e;
     if (d == 64)
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64>, dim3(grid), dim3(npa::KCfg<64>::kThreads), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, false>, dim3(grid), dim3(npa::KCfg<64>::kThreads), args,
                              npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
     else
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128>, dim3(grid), dim3(npa::KCfg<128>::kThreads), args,
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, false>, dim3(grid), dim3(npa::KCfg<128>::kThreads), args,
                              npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
     return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Global-token queries (text-query half of joint attention)
+// ---------------------------------------------------------------------------
+struct GqPlan {
+    int kc_log2, kr, n_blocks, n_qblocks, base_units, splits;
+    size_t split_bytes;  // workspace bytes per key-range split
+};
+
+GqPlan plan_gq(int B, int heads, int H, int W, int d, int G, int sm_count) {
+    GqPlan pl;
+    const Geo g{H, W, H, W, 0, 0};
+    pl.kc_log2 = choose_kc_log2(g);
+    pl.kr = 128 >> pl.kc_log2;
+    pl.n_blocks = ((W + (1 << pl.kc_log2) - 1) >> pl.kc_log2) * ((H + pl.kr - 1) / pl.kr) + (G + 127) / 128;
+    const int tiles = (G + 127) / 128;
+    pl.n_qblocks = (tiles + 1) / 2;
+    pl.base_units = B * heads * pl.n_qblocks;
+    // split the key range until the units roughly fill the GPU once
+    int s = (sm_count + pl.base_units / 2) / pl.base_units;
+    if (s < 1) s = 1;
+    if (s > 16) s = 16;
+    if (s > pl.n_blocks) s = pl.n_blocks;
+    pl.splits = s;
+    pl.split_bytes = (size_t)B * heads * G * (d + 2) * sizeof(float);
+    return pl;
+}
+
+npa_status launch_gq(const void *gq, const void *k, const void *v, const void *gk, const void *gv, void *go, int B,
+                     int heads, int H, int W, int d, int G, float *o_part, float *ml, int splits, int sm_count,
+                     npa_stream_t stream) {
+    const GqPlan pl = plan_gq(B, heads, H, W, d, G, sm_count);
+    FwdParams prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.o = go;
+    prm.H = H;
+    prm.W = W;
+    prm.G = G;
+    prm.Ph = H;
+    prm.Pw = W;
+    prm.nPh = prm.nPw = 1;
+    prm.kc_log2 = pl.kc_log2;
+    prm.kr = pl.kr;
+    prm.n_qblocks = pl.n_qblocks;
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+    prm.wait_limit_ns = kWaitLimitNs;
+    prm.BH = B * heads;
+    prm.n_splits = splits;
+    prm.gq_tiles = (G + 127) / 128;
+    prm.o_part = o_part;
+    prm.ml = ml;
+    const long long units = (long long)prm.BH * pl.n_qblocks * splits;
+    if (units > INT_MAX / 2) return NPA_ERR_UNSUPPORTED;
+    prm.n_units = (int)units;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)prm.BH};
+    const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)W * d * 2, (cuuint64_t)H * W * d * 2};
+    const cuuint32_t kbox[4] = {64, (cuuint32_t)(1 << pl.kc_log2), (cuuint32_t)pl.kr, 1};
+    const cuuint64_t gdims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)prm.BH};
+    const cuuint64_t gstrides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
+    const cuuint32_t gbox[3] = {64, 128, 1};
+    if (!encode(&prm.tm_k, k, 4, dims, strides, kbox) || !encode(&prm.tm_v, v, 4, dims, strides, kbox) ||
+        !encode(&prm.tm_gk, gk, 3, gdims, gstrides, gbox) || !encode(&prm.tm_gv, gv, 3, gdims, gstrides, gbox) ||
+        !encode(&prm.tm_gq, gq, 3, gdims, gstrides, gbox))
+        return NPA_ERR_CUDA;
+    const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);
+    void *args[1] = {&prm};
+    cudaError_t e;
+    if (d == 64)
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, true>, dim3(grid), dim3(npa::KCfg<64>::kThreads),
+                             args, npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
+    else
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, true>, dim3(grid),
+                             dim3(npa::KCfg<128>::kThreads), args, npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
+    if (e != cudaSuccess) return NPA_ERR_CUDA;
+    if (splits > 1) {
+        const int rows = prm.BH * G;
+        const float *op = o_part, *mlp = ml;
+        __nv_bfloat16 *gop = static_cast<__nv_bfloat16 *>(go);
+        int ns = splits, nr = rows;
+        void *cargs[5] = {&op, &mlp, &gop, &ns, &nr};
+        const dim3 cgrid((unsigned)((rows + 7) / 8));
+        if (d == 64)
+            e = cudaLaunchKernel((const void *)npa::gq_combine_kernel<64>, cgrid, dim3(256), cargs, 0,
+                                 (cudaStream_t)stream);
+        else
+            e = cudaLaunchKernel((const void *)npa::gq_combine_kernel<128>, cgrid, dim3(256), cargs, 0,
+                                 (cudaStream_t)stream);
+        if (e != cudaSuccess) return NPA_ERR_CUDA;
+    }
+    return NPA_OK;
+}
+
+npa_status validate_gq(const void *gq, const void *k, const void *v, const void *gk, const void *gv, void *go,
+                       int B, int heads, int H, int W, int d, int G) {
+    if (!gq || !k || !v || !gk || !gv || !go) return NPA_ERR_INVALID_ARG;
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || G < 1) return NPA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return NPA_ERR_UNSUPPORTED;
+    if (!aligned16(gq) || !aligned16(k) || !aligned16(v) || !aligned16(gk) || !aligned16(gv) || !aligned16(go))
+        return NPA_ERR_MISALIGNED;
+    const long long N = (long long)H * W, BH = (long long)B * heads;
+    if (N * d * 2 >= (1LL << 40) || BH > INT_MAX / 64 || N > INT_MAX || (long long)G * d * 2 >= (1LL << 40) ||
+        BH * G > INT_MAX / 2)
+        return NPA_ERR_UNSUPPORTED;
+    const size_t gbytes = (size_t)(BH * G * d * 2), ibytes = (size_t)(BH * N * d * 2);
+    if (overlaps(go, gbytes, gq, gbytes) || overlaps(go, gbytes, gk, gbytes) || overlaps(go, gbytes, gv, gbytes) ||
+        overlaps(go, gbytes, k, ibytes) || overlaps(go, gbytes, v, ibytes))
+        return NPA_ERR_INVALID_ARG;
+    return NPA_OK;
 }
 
 int neighbor_rows(int s, double p) {
@@ -352,6 +466,39 @@ npa_status pcpp_attention_fwd_stale(const void *q, const void *k, const void *v,
     const int s = H / n_strips;
     const Geo g{H, W, s, W, neighbor_rows(s, p), 0};
     return launch(q, k, v, k_stale, v_stale, o, B, heads, d, g, G, global_kv, strip_begin, strip_count, stream);
+}
+
+size_t npa_global_query_workspace_size(int B, int heads, int H, int W, int d, int G) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || G < 1 || (d != 64 && d != 128)) return 0;
+    int dev = 0, sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    const GqPlan pl = plan_gq(B, heads, H, W, d, G, sm);
+    return pl.splits > 1 ? (size_t)pl.splits * pl.split_bytes : 0;
+}
+
+npa_status npa_global_query_attention_fwd(const void *gq, const void *k, const void *v, const void *gk,
+                                          const void *gv, void *go, int B, int heads, int H, int W, int d, int G,
+                                          void *workspace, size_t workspace_bytes, npa_stream_t stream) {
+    npa_status st = validate_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G);
+    if (st != NPA_OK) return st;
+    if (workspace && !aligned16(workspace)) return NPA_ERR_MISALIGNED;
+    int sm_count = 0;
+    st = ensure_ready(&sm_count);
+    if (st != NPA_OK) return st;
+    const GqPlan pl = plan_gq(B, heads, H, W, d, G, sm_count);
+    // as many splits as planned and as the workspace holds (one needs none)
+    int splits = workspace ? (int)(workspace_bytes / pl.split_bytes) : 1;
+    if (splits > pl.splits) splits = pl.splits;
+    if (splits < 2) splits = 1;
+    float *o_part = static_cast<float *>(workspace);
+    float *ml = splits > 1 ? o_part + (size_t)splits * B * heads * G * d : nullptr;
+    if (splits > 1) {
+        const size_t wsz = (size_t)splits * pl.split_bytes;
+        const size_t gbytes = (size_t)B * heads * G * d * 2;
+        if (overlaps(workspace, wsz, go, gbytes) || overlaps(workspace, wsz, gq, gbytes)) return NPA_ERR_INVALID_ARG;
+    }
+    return launch_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G, o_part, ml, splits, sm_count, stream);
 }
 
 int pcpp_neighbor_rows(int strip_rows, double p) { return neighbor_rows(strip_rows, p); }

@@ -115,7 +115,9 @@ struct KCfg {
 // Phases are counted across units: gb = key blocks processed so far by this
 // CTA (one S and one P per tile per block), uq = units processed so far.
 // ---------------------------------------------------------------------------
+template <bool GQ>
 __device__ __forceinline__ bool unit_has_work(const FwdParams &p, const Work &w) {
+    if (GQ) return w.tile0 < p.gq_tiles && w.je > w.jb;
     return q_tile_valid(p, w, w.tile0) || q_tile_valid(p, w, w.tile0 + 1);
 }
 
@@ -141,7 +143,7 @@ __device__ __forceinline__ void load_block(const FwdParams &p, const Work &w, in
     }
 }
 
-template <int D>
+template <int D, bool GQ>
 __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
     const uint64_t lim = p.wait_limit_ns;
@@ -156,12 +158,13 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
         sm100::tma_prefetch_desc(&p.tm_ks);
         sm100::tma_prefetch_desc(&p.tm_vs);
     }
-    const uint32_t q_bytes = uint32_t(C::kChunks * p.qc * p.qr * 128);
+    if (GQ) sm100::tma_prefetch_desc(&p.tm_gq);
+    const uint32_t q_bytes = GQ ? uint32_t(C::kChunks * 128 * 128) : uint32_t(C::kChunks * p.qc * p.qr * 128);
     int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q pairs issued
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-        const Work w = decode_work(p, unit);
-        if (!unit_has_work(p, w)) continue;
+        const Work w = decode<GQ>(p, unit);
+        if (!unit_has_work<GQ>(p, w)) continue;
         // the previous unit's last S products must be done with the Q buffer
         if (uq > 0 && !sm100::mbar_wait(&bars[C::bQEmpty], (uq - 1) & 1, lim)) {
             ok = false;
@@ -170,15 +173,22 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
         sm100::mbar_arrive_expect_tx(&bars[C::bQFull], 2 * q_bytes);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-            int row0, col0;
-            q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
+            if (GQ) {
 #pragma unroll
-            for (int c = 0; c < C::kChunks; ++c)
-                sm100::tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
-                                   &bars[C::bQFull], c * 64, col0, row0, w.bh);
+                for (int c = 0; c < C::kChunks; ++c)
+                    sm100::tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_gq,
+                                       &bars[C::bQFull], c * 64, (w.tile0 + t) * 128, w.bh);
+            } else {
+                int row0, col0;
+                q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
+#pragma unroll
+                for (int c = 0; c < C::kChunks; ++c)
+                    sm100::tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                                       &bars[C::bQFull], c * 64, col0, row0, w.bh);
+            }
         }
         ++uq;
-        for (int j = 0; j < w.n_blocks; ++j) {
+        for (int j = w.jb; j < w.je; ++j) {
             if (*abort_flag) {
                 ok = false;
                 break;
@@ -265,7 +275,7 @@ __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
 // independently. This one issues S_0(j), S_1(j) as soon as the softmax warps
 // hold S(j-1) in registers; the first S of a unit also overlaps the previous
 // unit's last P.V products and epilogue.
-template <int D>
+template <int D, bool GQ>
 __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                           volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
@@ -274,11 +284,11 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
     int gb = 0, uq = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-        const Work w = decode_work(p, unit);
-        if (!unit_has_work(p, w)) continue;
+        const Work w = decode<GQ>(p, unit);
+        if (!unit_has_work<GQ>(p, w)) continue;
         ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
-        for (int j = 0; ok && j < w.n_blocks; ++j, ++gb) {
+        for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
             if (*abort_flag) {
                 ok = false;
                 break;
@@ -305,7 +315,7 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
 }
 
 // d = 64: the P.V products, O_q(j) += P_q(j) V(j) as each P_q(j) arrives.
-template <int D>
+template <int D, bool GQ>
 __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                            volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
@@ -314,9 +324,9 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
     int gb = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-        const Work w = decode_work(p, unit);
-        if (!unit_has_work(p, w)) continue;
-        for (int j = 0; ok && j < w.n_blocks; ++j, ++gb) {
+        const Work w = decode<GQ>(p, unit);
+        if (!unit_has_work<GQ>(p, w)) continue;
+        for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
             if (*abort_flag) {
                 ok = false;
                 break;
@@ -327,7 +337,7 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
                 ok = sm100::mbar_wait(&bars[C::bPFull + q], gb & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > 0);
+                issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > w.jb);
                 sm100::tc_commit(&bars[C::bPFree + q]);
             }
             if (ok) sm100::tc_commit(&bars[C::bVEmpty + s]);
@@ -343,7 +353,7 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
 
 // d = 128 (P aliases S): one warp issues everything, PV_q(j-1) before S_q(j)
 // for each tile, so that the completion of S_q(j) also implies PV_q(j-1).
-template <int D>
+template <int D, bool GQ>
 __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                         volatile uint32_t *abort_flag) {
     using C = KCfg<D>;
@@ -352,9 +362,9 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
     int gb = 0, uq = 0;  // gb: global index of block j = 0 of the current unit
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-        const Work w = decode_work(p, unit);
-        if (!unit_has_work(p, w)) continue;
-        const int n = w.n_blocks;
+        const Work w = decode<GQ>(p, unit);
+        if (!unit_has_work<GQ>(p, w)) continue;
+        const int n = w.je - w.jb;  // blocks of this unit, counted from its first
         ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
         sm100::tc_fence_after();
@@ -484,7 +494,7 @@ __device__ __forceinline__ float exp_block(const float (&s)[128], float c, float
     return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
-template <int D>
+template <int D, bool GQ>
 __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
                             int q) {
     using C = KCfg<D>;
@@ -500,17 +510,20 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
     int gb = 0;  // global index (across units) of the current block
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
-    const Work w = decode_work(p, unit);
-    if (!unit_has_work(p, w)) continue;
-    const int n_blocks = w.n_blocks;
+    const Work w = decode<GQ>(p, unit);
+    if (!unit_has_work<GQ>(p, w)) continue;
     // window block coordinates, advanced without divisions: column block,
     // first row of the current band, end of the band's row segment
     int btc = 0, brow = w.seg[0], bend = w.seg[1];
     if (brow >= bend) bend = w.seg[2];
+    if (GQ && w.jb > 0 && w.jb < w.n_win) {  // a key-range split starts inside the (one-segment) grid
+        btc = w.jb % w.wtc;
+        brow = (w.jb / w.wtc) * p.kr;
+    }
     float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
     float R_prev = -INFINITY;  // reference that O and l are currently expressed in
     float l = 0.f;
-    for (int j = 0; j < n_blocks; ++j, ++gb) {
+    for (int j = w.jb; j < w.je; ++j, ++gb) {
         if (!warp_wait(&bars[C::bSFull + q], gb & 1, lim)) {
             ok = false;
             break;
@@ -571,7 +584,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             if (lane0) sm100::mbar_arrive(&bars[C::bTurn + (q ^ 1)]);
         }
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
-        if (C::kSeparateP && j > 0) {
+        if (C::kSeparateP && j > w.jb) {
             // PV_q(j-1) must be done before O is rescaled or P_q overwritten
             if (!warp_wait(&bars[C::bPFree + q], (gb - 1) & 1, lim)) {
                 ok = false;
@@ -579,7 +592,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
             sm100::tc_fence_after();
         }
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (j > w.jb && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
@@ -602,13 +615,39 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
     // epilogue: O / l -> bf16 -> the query's token position
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const int t = w.tile0 + q;
-    int row0, col0;
-    q_tile_origin(p, w, t, &row0, &col0);
-    const int rr = row / p.qc, cc = row - rr * p.qc;
-    const int grow = row0 + rr, gcol = col0 + cc;
-    const bool valid = t < p.tiles_c * p.tiles_r && row < p.qc * p.qr && grow < w.pr1 && gcol < w.pc1;
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) +
-                                           ((size_t)w.bh * p.H * p.W + (size_t)grow * p.W + gcol) * D);
+    bool valid;
+    size_t out_row;
+    if (GQ) {
+        const int g = t * 128 + row;
+        valid = t < p.gq_tiles && g < p.G;
+        out_row = (size_t)w.bh * p.G + g;
+        if (p.n_splits > 1) {
+            // a key-range split: unnormalised O with its reference maximum and row sum
+            const size_t prow = (size_t)w.split * p.BH * p.G + out_row;
+            float4 *part = reinterpret_cast<float4 *>(p.o_part + prow * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                sm100::tmem_ld32(tO + c * 32, o);
+                if (valid) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        part[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                                      __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+                }
+            }
+            if (valid) *reinterpret_cast<float2 *>(p.ml + prow * 2) = make_float2(R_prev, l);
+            continue;
+        }
+    } else {
+        int row0, col0;
+        q_tile_origin(p, w, t, &row0, &col0);
+        const int rr = row / p.qc, cc = row - rr * p.qc;
+        const int grow = row0 + rr, gcol = col0 + cc;
+        valid = t < p.tiles_c * p.tiles_r && row < p.qc * p.qr && grow < w.pr1 && gcol < w.pc1;
+        out_row = (size_t)w.bh * p.H * p.W + (size_t)grow * p.W + gcol;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D);
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
@@ -635,7 +674,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool GQ>
 __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = KCfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -680,17 +719,17 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
     if (warp >= 8) {
         sm100::setmaxnreg_dec<C::kRegsCtl>();
         if ((threadIdx.x & 31) == 0) {
-            if (warp == 8) run_producer<D>(p, smem, bars, abort_flag);
+            if (warp == 8) run_producer<D, GQ>(p, smem, bars, abort_flag);
             if (C::kSeparateP) {
-                if (warp == 9) run_mma_s<D>(p, smem, bars, tmem, abort_flag);
-                if (warp == 10) run_mma_pv<D>(p, smem, bars, tmem, abort_flag);
+                if (warp == 9) run_mma_s<D, GQ>(p, smem, bars, tmem, abort_flag);
+                if (warp == 10) run_mma_pv<D, GQ>(p, smem, bars, tmem, abort_flag);
             } else if (warp == 9) {
-                run_mma<D>(p, smem, bars, tmem, abort_flag);
+                run_mma<D, GQ>(p, smem, bars, tmem, abort_flag);
             }
         }
     } else {
         sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D>(p, bars, tmem, abort_flag, warp >> 2);
+        run_softmax<D, GQ>(p, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();
@@ -700,6 +739,37 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
         __syncwarp();
         sm100::tmem_dealloc(tmem, C::kTmemCols);
     }
+}
+
+// Merges the key-range splits of global-token queries: one warp per query
+// row; with m* the largest split reference, O = sum_s 2^(m_s - m*) O_s /
+// sum_s 2^(m_s - m*) l_s, rounded to bf16.
+template <int D>
+__global__ void __launch_bounds__(256) gq_combine_kernel(const float *__restrict__ o_part,
+                                                         const float *__restrict__ ml, __nv_bfloat16 *go,
+                                                         int n_splits, int rows) {
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= rows) return;
+    const int lane = threadIdx.x & 31;
+    constexpr int kPer = D / 32;  // channels per lane
+    float mstar = -INFINITY;
+    for (int s = 0; s < n_splits; ++s) mstar = fmaxf(mstar, ml[((size_t)s * rows + r) * 2]);
+    float acc[kPer];
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+    float L = 0.f;
+    for (int s = 0; s < n_splits; ++s) {
+        const size_t pr = (size_t)s * rows + r;
+        const float m = ml[pr * 2];
+        const float wgt = (m == -INFINITY) ? 0.f : sm100::ex2_approx(m - mstar);
+        L += wgt * ml[pr * 2 + 1];
+#pragma unroll
+        for (int c = 0; c < kPer; ++c) acc[c] += wgt * o_part[pr * D + lane * kPer + c];
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint32_t *dst = reinterpret_cast<uint32_t *>(go + (size_t)r * D + lane * kPer);
+#pragma unroll
+    for (int c = 0; c < kPer; c += 2) dst[c / 2] = sm100::pack_bf16x2(acc[c] * inv, acc[c + 1] * inv);
 }
 
 // One block, one thread waiting on a barrier nothing arrives at: exercises the

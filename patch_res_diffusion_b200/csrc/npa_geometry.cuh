@@ -35,6 +35,7 @@ struct FwdParams {
     CUtensorMap tm_gv;
     CUtensorMap tm_ks;  // previous step's K / V for the borrowed rows (two_source only)
     CUtensorMap tm_vs;
+    CUtensorMap tm_gq;  // global-token queries: 3D {d, G, B*heads}, box {64, 128, 1}
     void *o;            // bf16 [B, heads, H*W, d]
     int H, W, G;
     int Ph, Pw, mh, mw;
@@ -48,6 +49,10 @@ struct FwdParams {
     int n_units;                     // work units in execution order
     int two_source;                  // 1: rows outside the patch come from tm_ks / tm_vs
     int patch_begin, patch_count;    // patches computed (natural order when n_perm == 0)
+    int n_splits;                    // global-token queries: key-range splits per query tile pair
+    int gq_tiles;                    // global-token queries: ceil(G / 128)
+    float *o_part;                   // splits > 1: [n_splits][B*heads][G][d] unnormalised O
+    float *ml;                       // splits > 1: [n_splits][B*heads][G][2] reference max, row sum
     int n_perm;                      // entries of patch_order (0: natural order)
     unsigned short patch_order[kMaxPatchOrder];  // patches by decreasing window area
 };
@@ -65,6 +70,8 @@ struct Work {
     int tile0;                // first query tile (of two) within the patch
     int wtc;                  // window blocks along the columns
     int n_win, n_blocks;      // window blocks, window + global blocks
+    int jb, je;               // the unit's key blocks [jb, je) (a key-range split)
+    int split;
 };
 
 // Where key block j (< n_win) of a unit lies: first row and column of its box,
@@ -114,7 +121,43 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     w.nb01 = w.nb0 + w.wtc * cdiv_(w.seg[2] - w.seg[1], p.kr);
     w.n_win = w.nb01 + w.wtc * cdiv_(w.seg[3] - w.seg[2], p.kr);
     w.n_blocks = w.n_win + cdiv_(p.G, 128);
+    w.jb = 0;
+    w.je = w.n_blocks;
+    w.split = 0;
     return w;
+}
+
+// Global-token queries (the text-query half of joint attention): a unit is
+// (batch*head, key-range split, pair of 128-token query tiles); the window is
+// the whole grid followed by the global tokens, and split s covers key
+// blocks [s*n/S, (s+1)*n/S).
+__host__ __device__ inline Work decode_work_gq(const FwdParams &p, int unit) {
+    Work w;
+    const int qb = unit % p.n_qblocks;
+    const int rest = unit / p.n_qblocks;
+    w.split = rest % p.n_splits;
+    w.bh = rest / p.n_splits;
+    w.pr0 = w.pc0 = 0;
+    w.pr1 = p.H;
+    w.pc1 = p.W;
+    w.wr0 = w.wc0 = 0;
+    w.wr1 = p.H;
+    w.wc1 = p.W;
+    w.seg[0] = w.seg[1] = 0;
+    w.seg[2] = w.seg[3] = p.H;
+    w.tile0 = 2 * qb;
+    w.wtc = cdiv_(p.W, 1 << p.kc_log2);
+    w.nb0 = 0;
+    w.nb01 = w.n_win = w.wtc * cdiv_(p.H, p.kr);
+    w.n_blocks = w.n_win + cdiv_(p.G, 128);
+    w.jb = (int)((long long)w.split * w.n_blocks / p.n_splits);
+    w.je = (int)((long long)(w.split + 1) * w.n_blocks / p.n_splits);
+    return w;
+}
+
+template <bool GQ>
+__host__ __device__ inline Work decode(const FwdParams &p, int unit) {
+    return GQ ? decode_work_gq(p, unit) : decode_work(p, unit);
 }
 
 __host__ __device__ inline BlockGeom block_geom(const FwdParams &p, const Work &w, int j) {

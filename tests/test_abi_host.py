@@ -159,3 +159,17 @@ def test_stale_entry_point_validation(L):
     assert _stale(L, H=9) == npa.NPA_ERR_INVALID_ARG
     assert _stale(L, p=2.0) == npa.NPA_ERR_INVALID_ARG
     assert _stale(L, d=96) == npa.NPA_ERR_UNSUPPORTED
+
+
+def test_global_query_validation(L):
+    f = lambda gq=A, k=B_, v=C_, gk=0x30000000, gv=0x50000000, go=O_, G=5, d=64, ws=None: \
+        L.npa_global_query_attention_fwd(gq, k, v, gk, gv, go, 1, 1, 8, 8, d, G, ws, 0, None)
+    assert f(gq=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(gk=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(G=0) == npa.NPA_ERR_INVALID_ARG
+    assert f(d=96) == npa.NPA_ERR_UNSUPPORTED
+    assert f(go=O_ + 4) == npa.NPA_ERR_MISALIGNED
+    assert f(go=A) == npa.NPA_ERR_INVALID_ARG          # output overlaps the queries
+    assert f(ws=0x70000008) == npa.NPA_ERR_MISALIGNED
+    assert L.npa_global_query_workspace_size(1, 1, 8, 8, 96, 5) == 0
+    assert L.npa_global_query_workspace_size(1, 1, 8, 8, 64, 0) == 0
