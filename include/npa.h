@@ -37,8 +37,9 @@
  * Ownership and ordering: the caller owns every buffer. Calls are
  * asynchronous and ordered on `stream` (NULL = the legacy default stream);
  * buffers must stay valid until the stream reaches the call. The compute
- * entry points allocate no device memory; the library's only device state is
- * one status word per device (see npa_device_status). Host-side state is
+ * entry points allocate no device memory; the library's device state is one
+ * status word per device (see npa_device_status) and the fixed scratch array
+ * of npa_global_query_attention_fwd_noalloc. Host-side state is
  * limited to per-device capability checks and kernel attributes, set up under
  * a lock on first use, so the entry points are safe to call from several host
  * threads.
@@ -129,6 +130,28 @@ npa_status pcpp_attention_fwd_stale(const void *q, const void *k, const void *v,
 npa_status npa_global_query_attention_fwd(const void *gq, const void *k, const void *v, const void *gk,
                                           const void *gv, void *go, int B, int heads, int H, int W, int d,
                                           int G, void *workspace, size_t workspace_bytes, npa_stream_t stream);
+
+/* npa_global_query_attention_fwd for callers that cannot hand the library
+ * device memory: for example a plugin whose host framework owns every device
+ * allocation and exposes no allocator to it, or a service that forbids
+ * device allocation after start-up because cudaMalloc can synchronise the
+ * device and stall other work. The pages have no counterpart to this; it
+ * is a deployment variant of the same computation.
+ * The key-range split partials go to a fixed 16 MiB array inside the library
+ * (allocated when the library is loaded, held by every GPU that loads it
+ * until the process exits); nothing is allocated per call. The array must
+ * hold at least two partial results, 2 * B * heads * G * (d + 2) * 4 bytes
+ * <= 16 MiB, else the call returns NPA_ERR_UNSUPPORTED before touching the
+ * device; the split count is also limited by the array. The
+ * first call on each device looks up the array's device address (with that
+ * device current) and should come before any stream capture. Every call
+ * shares the array and overwrites it; nothing in it needs to start at zero.
+ * Calls that overlap on the GPU (other streams, other host threads) race on
+ * the array: order them on one stream. Other arguments, results and errors
+ * as for npa_global_query_attention_fwd. */
+npa_status npa_global_query_attention_fwd_noalloc(const void *gq, const void *k, const void *v, const void *gk,
+                                                  const void *gv, void *go, int B, int heads, int H, int W,
+                                                  int d, int G, npa_stream_t stream);
 
 /* Workspace bytes npa_global_query_attention_fwd uses for its full split
  * count on the current device (0: no split needed, or invalid arguments). */

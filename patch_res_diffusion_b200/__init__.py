@@ -25,7 +25,8 @@ __all__ = [
     "pcpp_attention_fwd", "pcpp_neighbor_rows", "npa_useful_flops", "pcpp_useful_flops",
     "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string", "npa_attention",
     "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "npa_global_query_attention_fwd",
-    "npa_global_query_workspace_size", "global_query_attention", "EXPORTED_SYMBOLS",
+    "npa_global_query_workspace_size", "npa_global_query_attention_fwd_noalloc", "global_query_attention",
+    "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
@@ -41,6 +42,7 @@ EXPORTED_SYMBOLS = (
     "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_attention_fwd_stale", "pcpp_neighbor_rows", "npa_useful_flops",
     "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
     "npa_global_query_attention_fwd", "npa_global_query_workspace_size",
+    "npa_global_query_attention_fwd_noalloc",
 )
 
 
@@ -74,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.pcpp_attention_fwd_stale.restype = i
         L.npa_global_query_attention_fwd.argtypes = [vp] * 6 + [i] * 6 + [vp, ctypes.c_size_t, vp]
         L.npa_global_query_attention_fwd.restype = i
+        L.npa_global_query_attention_fwd_noalloc.argtypes = [vp] * 6 + [i] * 6 + [vp]
+        L.npa_global_query_attention_fwd_noalloc.restype = i
         L.npa_global_query_workspace_size.argtypes = [i] * 6
         L.npa_global_query_workspace_size.restype = ctypes.c_size_t
         L.pcpp_neighbor_rows.argtypes = [i, d]
@@ -159,6 +163,15 @@ def npa_global_query_attention_fwd(gq, k, v, gk, gv, go, B: int, heads: int, H: 
                                                 H, W, d, G, _ptr(workspace), int(workspace_bytes),
                                                 _stream(stream)),
            "npa_global_query_attention_fwd")
+
+
+def npa_global_query_attention_fwd_noalloc(gq, k, v, gk, gv, go, B: int, heads: int, H: int, W: int, d: int,
+                                           G: int, stream=None) -> None:
+    """C ``npa_global_query_attention_fwd_noalloc``: the same computation with
+    the split partials in the library's fixed device array (no caller memory)."""
+    _check(lib().npa_global_query_attention_fwd_noalloc(_ptr(gq), _ptr(k), _ptr(v), _ptr(gk), _ptr(gv), _ptr(go),
+                                                        B, heads, H, W, d, G, _stream(stream)),
+           "npa_global_query_attention_fwd_noalloc")
 
 
 def npa_global_query_workspace_size(B, heads, H, W, d, G) -> int:

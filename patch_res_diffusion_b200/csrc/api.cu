@@ -411,6 +411,18 @@ npa_status validate_gq(const void *gq, const void *k, const void *v, const void 
     return NPA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Fixed scratch for npa_global_query_attention_fwd_noalloc: the key-range
+// split partials live in this file-scope device array instead of caller
+// memory. Every GPU that loads the library holds it until the process exits.
+// In host code g_noalloc_scratch only stands for the symbol; its device
+// address is fetched once per device with cudaGetSymbolAddress (with that
+// device current) and passed to the kernels.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void *g_noalloc_addr[kMaxDevices] = {};
+
 int neighbor_rows(int s, double p) {
     if (s < 1 || !(p >= 0.0) || !(p <= 1.0)) return -1;
     int r = (int)std::ceil(p * (double)s - 1e-9);
@@ -498,6 +510,41 @@ npa_status npa_global_query_attention_fwd(const void *gq, const void *k, const v
         const size_t gbytes = (size_t)B * heads * G * d * 2;
         if (overlaps(workspace, wsz, go, gbytes) || overlaps(workspace, wsz, gq, gbytes)) return NPA_ERR_INVALID_ARG;
     }
+    return launch_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G, o_part, ml, splits, sm_count, stream);
+}
+
+npa_status npa_global_query_attention_fwd_noalloc(const void *gq, const void *k, const void *v, const void *gk,
+                                                  const void *gv, void *go, int B, int heads, int H, int W, int d,
+                                                  int G, npa_stream_t stream) {
+    npa_status st = validate_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G);
+    if (st != NPA_OK) return st;
+    // the array must hold at least two partial results (the smallest split);
+    // the limit does not depend on the device, so it is checked first
+    const size_t per_split = (size_t)B * heads * G * (d + 2) * sizeof(float);
+    if (2 * per_split > kNoAllocScratchBytes) return NPA_ERR_UNSUPPORTED;
+    int sm_count = 0;
+    st = ensure_ready(&sm_count);
+    if (st != NPA_OK) return st;
+    const GqPlan pl = plan_gq(B, heads, H, W, d, G, sm_count);
+    int splits = 1;
+    if (pl.splits > 1) {
+        splits = (int)(kNoAllocScratchBytes / per_split);
+        if (splits > pl.splits) splits = pl.splits;
+    }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return NPA_ERR_CUDA;
+    void *base = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_noalloc_addr[dev]) {
+            void *ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return NPA_ERR_CUDA;
+            g_noalloc_addr[dev] = ptr;
+        }
+        base = g_noalloc_addr[dev];
+    }
+    float *o_part = splits > 1 ? static_cast<float *>(base) : nullptr;
+    float *ml = splits > 1 ? o_part + (size_t)splits * B * heads * G * d : nullptr;
     return launch_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G, o_part, ml, splits, sm_count, stream);
 }
 
