@@ -193,41 +193,6 @@ npa_status validate_common(const void *q, const void *k, const void *v, void *o,
     return NPA_OK;
 }
 
-// Patches ordered by decreasing number of key blocks (ties: natural order),
-// so a persistent CTA's last units are its cheapest.
-void order_patches(const Geo &g, FwdParams &prm) {
-    const int np = prm.patch_count;
-    if (np > npa::kMaxPatchOrder) {
-        prm.n_perm = 0;
-        return;
-    }
-    const int kc = 1 << prm.kc_log2;
-    int cost[npa::kMaxPatchOrder];  // indexed by position in the patch range
-    for (int i = 0; i < np; ++i) {
-        const int patch = prm.patch_begin + i;
-        const int pi = patch / prm.nPw, pj = patch % prm.nPw;
-        const int r0 = pi * g.Ph, r1 = r0 + g.Ph < g.H ? r0 + g.Ph : g.H;
-        const int c0 = pj * g.Pw, c1 = c0 + g.Pw < g.W ? c0 + g.Pw : g.W;
-        const int wh = (r1 + g.mh < g.H ? r1 + g.mh : g.H) - (r0 - g.mh > 0 ? r0 - g.mh : 0);
-        const int ww = (c1 + g.mw < g.W ? c1 + g.mw : g.W) - (c0 - g.mw > 0 ? c0 - g.mw : 0);
-        cost[i] = ((ww + kc - 1) / kc) * ((wh + prm.kr - 1) / prm.kr);
-    }
-    unsigned short idx[npa::kMaxPatchOrder];
-    for (int i = 0; i < np; ++i) idx[i] = (unsigned short)i;
-    // insertion sort, stable, descending cost (np <= 256)
-    for (int i = 1; i < np; ++i) {
-        const unsigned short x = idx[i];
-        int j = i - 1;
-        while (j >= 0 && cost[idx[j]] < cost[x]) {
-            idx[j + 1] = idx[j];
-            --j;
-        }
-        idx[j + 1] = x;
-    }
-    for (int i = 0; i < np; ++i) prm.patch_order[i] = (unsigned short)(prm.patch_begin + idx[i]);
-    prm.n_perm = np;
-}
-
 // ks / vs (both or neither): previous-step keys/values for the rows of a
 // window outside its patch. [patch_begin, patch_begin + patch_count): the
 // patches computed, in natural numbering; patch_count < 0 means all.
@@ -269,7 +234,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     const int BH = B * heads;
     prm.BH = BH;
     prm.n_units = (int)units;
-    order_patches(g, prm);
+    npa::order_patches(prm);
     // persistent grid: one CTA per multiprocessor (shared memory and TMEM
     // admit one), each walking every gridDim.x-th unit
     const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);

@@ -1,0 +1,74 @@
+"""The persistent kernel's work-unit order (host arithmetic, no GPU): every
+(batch*head, patch, query-tile pair) of the computed patch range is decoded
+exactly once, cheapest units last, for NPA and PCPP geometries with ragged
+patches, patch ranges and more cost classes than the class table holds."""
+import os
+import shutil
+import subprocess
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+@pytest.fixture(scope="module")
+def checker(tmp_path_factory):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    exe = str(tmp_path_factory.mktemp("sched") / "unit_schedule_check")
+    subprocess.run([nvcc, "-std=c++17", "-O1", "-Wno-deprecated-gpu-targets", "-o", exe, os.path.join(HERE, "unit_schedule_check.cu")],
+                   check=True, capture_output=True)
+    return exe
+
+
+def run(exe, *args):
+    out = subprocess.run([exe, *map(str, args)], capture_output=True, text=True)
+    assert out.returncode == 0, out.stdout + out.stderr
+    f = out.stdout.split()
+    return {"units": int(f[2]), "ordered": int(f[4]), "classes": int(f[6]), "wave_heads": int(f[8])}
+
+
+# BH, H, W, Ph, Pw, mh, mw, kc_log2, n_qblocks, patch_begin, patch_count
+CASES = {
+    "npa_sdxl_4096": (20, 256, 256, 64, 64, 32, 32, 5, 16, 0, -1),
+    "npa_flux_4096": (24, 256, 256, 64, 64, 32, 32, 5, 16, 0, -1),
+    "npa_sdxl_2048": (20, 128, 128, 64, 64, 32, 32, 5, 16, 0, -1),
+    "ragged": (3, 40, 37, 16, 16, 5, 5, 4, 1, 0, -1),
+    "ragged_small_patches": (2, 100, 100, 9, 9, 3, 3, 3, 1, 0, -1),
+    "pcpp_4x32": (20, 128, 128, 32, 128, 8, 0, 7, 16, 0, -1),
+    "pcpp_strip_range": (4, 64, 64, 8, 64, 3, 0, 6, 2, 3, 4),
+    "npa_patch_range": (4, 64, 64, 16, 16, 4, 4, 4, 1, 3, 7),
+    "unordered": (2, 61, 59, 3, 4, 1, 2, 3, 1, 0, -1),        # 315 patches: natural order
+    "fifteen_classes": (2, 300, 300, 20, 20, 60, 60, 3, 1, 0, -1),
+    "too_many_classes": (2, 300, 300, 20, 20, 100, 100, 3, 1, 0, -1),  # ordered, no class table
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_every_unit_once_cheapest_last(checker, name):
+    r = run(checker, *CASES[name], 148)
+    a = CASES[name]
+    n_patches = ((a[1] + a[3] - 1) // a[3]) * ((a[2] + a[4] - 1) // a[4])
+    count = n_patches - a[9] if a[10] < 0 else a[10]
+    assert r["units"] == a[0] * count * a[8]
+
+
+def test_concurrent_units_share_heads(checker):
+    """SDXL 4096^2 (B2 h10, 4x4 patches of 64, margin 32): the windows fall in
+    3 cost classes, and the first 148 units (one per SM) cover only 3 of the
+    20 batch*heads, so their overlapping windows are shared in L2."""
+    r = run(checker, *CASES["npa_sdxl_4096"], 148)
+    assert r["classes"] == 3
+    assert r["wave_heads"] <= 3
+
+
+def test_fallbacks(checker):
+    """Past 256 patches the units run in natural patch order; past 16 cost
+    classes they keep the cost order but vary batch*head fastest."""
+    r = run(checker, *CASES["unordered"], 148)
+    assert r["ordered"] == 0 and r["classes"] == 0
+    r = run(checker, *CASES["fifteen_classes"], 148)
+    assert r["ordered"] == 225 and r["classes"] == 15
+    r = run(checker, *CASES["too_many_classes"], 148)
+    assert r["ordered"] == 225 and r["classes"] == 0

@@ -1,0 +1,70 @@
+// Host-only check of the persistent kernel's work-unit schedule: for one
+// geometry given on the command line it decodes every unit index and checks
+// that each (batch*head, patch, query-tile pair) of the patch range occurs
+// exactly once, that unit costs never increase along the order when an
+// order was built (at most kMaxPatchOrder patches), and prints the number of
+// ordered patches, the number of cost classes and the batch*head values the
+// first `wave` units touch. Built and run by test_unit_schedule.py.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <set>
+#include <vector>
+
+#include "../patch_res_diffusion_b200/csrc/npa_geometry.cuh"
+
+int main(int argc, char **argv) {
+    if (argc != 13) {
+        std::fprintf(stderr, "usage: BH H W Ph Pw mh mw kc_log2 n_qblocks patch_begin patch_count wave\n");
+        return 2;
+    }
+    int a[12];
+    for (int i = 0; i < 12; ++i) a[i] = std::atoi(argv[i + 1]);
+    npa::FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.BH = a[0];
+    p.H = a[1];
+    p.W = a[2];
+    p.Ph = a[3];
+    p.Pw = a[4];
+    p.mh = a[5];
+    p.mw = a[6];
+    p.kc_log2 = a[7];
+    p.kr = 128 >> p.kc_log2;
+    p.n_qblocks = a[8];
+    p.nPh = (p.H + p.Ph - 1) / p.Ph;
+    p.nPw = (p.W + p.Pw - 1) / p.Pw;
+    p.patch_begin = a[9];
+    p.patch_count = a[10] < 0 ? p.nPh * p.nPw - p.patch_begin : a[10];
+    const int wave = a[11];
+    p.n_units = p.BH * p.patch_count * p.n_qblocks;
+    npa::order_patches(p);
+    const int n_patches = p.nPh * p.nPw;
+    std::vector<int> seen((size_t)p.BH * n_patches * p.n_qblocks, 0);
+    int prev_cost = 1 << 30;
+    std::set<int> wave_bh;
+    for (int u = 0; u < p.n_units; ++u) {
+        const npa::Work w = npa::decode_work(p, u);
+        const int patch = (w.pr0 / p.Ph) * p.nPw + w.pc0 / p.Pw;
+        const int qb = w.tile0 / 2;
+        if (w.bh < 0 || w.bh >= p.BH || patch < p.patch_begin || patch >= p.patch_begin + p.patch_count ||
+            qb < 0 || qb >= p.n_qblocks) {
+            std::printf("FAIL unit %d decodes outside the range (bh %d patch %d pair %d)\n", u, w.bh, patch, qb);
+            return 1;
+        }
+        const int cost = npa::patch_cost(p, patch);
+        if (p.n_perm > 0 && cost > prev_cost) {
+            std::printf("FAIL unit %d cost %d after %d\n", u, cost, prev_cost);
+            return 1;
+        }
+        prev_cost = cost;
+        if (++seen[((size_t)w.bh * n_patches + patch) * p.n_qblocks + qb] != 1) {
+            std::printf("FAIL unit %d repeats (bh %d patch %d pair %d)\n", u, w.bh, patch, qb);
+            return 1;
+        }
+        if (u < wave) wave_bh.insert(w.bh);
+    }
+    std::printf("ok units %d ordered %d classes %d wave_heads %d\n", p.n_units, p.n_perm, p.n_cls,
+                (int)wave_bh.size());
+    return 0;
+}
