@@ -21,6 +21,16 @@ using npa::FwdParams;
 // below a millisecond).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Query tiles per CTA for image-token queries at d = 64: 2 (128-key blocks)
+// or, built with NPA_D64_TILES=3, three tiles on 64-key blocks (three softmax
+// warpgroups share the exponential unit; measured no faster). d = 128 and the
+// global-token queries always run two tiles on 128-key blocks.
+#ifndef NPA_D64_TILES
+#define NPA_D64_TILES 2
+#endif
+static_assert(NPA_D64_TILES == 2 || NPA_D64_TILES == 3, "NPA_D64_TILES");
+constexpr int kD64Tiles = NPA_D64_TILES;
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -34,6 +44,10 @@ struct DeviceState {
     int sm_count = 0;
 };
 DeviceState g_dev[kMaxDevices];
+
+bool set_smem(void (*kernel)(FwdParams), int bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
 
 // Resolves the tensor-map encoder and checks (once per device) that the
 // current device is an sm_100 part; sets the kernels' shared-memory limits.
@@ -62,15 +76,14 @@ npa_status ensure_ready(int *sm_count = nullptr) {
             return NPA_ERR_CUDA;
         if (major != 10 || minor != 0) {
             ds.status = NPA_ERR_UNSUPPORTED;
-        } else if (cudaFuncSetAttribute(npa::npa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        npa::KCfg<64>::kSmemBytes) != cudaSuccess ||
-                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128, false>,
-                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        npa::KCfg<128>::kSmemBytes) != cudaSuccess ||
-                   cudaFuncSetAttribute(npa::npa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        npa::KCfg<64>::kSmemBytes) != cudaSuccess ||
-                   cudaFuncSetAttribute(npa::npa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        npa::KCfg<128>::kSmemBytes) != cudaSuccess) {
+        } else if (
+#if NPA_D64_TILES == 3
+                   !set_smem(npa::npa_fwd_kernel<64, 3, 64, false>, npa::KCfg<64, 3, 64>::kSmemBytes) ||
+#endif
+                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, false>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
+                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, false>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
+                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
+                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, true>, npa::KCfg<128, 2, 128>::kSmemBytes)) {
             return NPA_ERR_CUDA;
         } else {
             ds.status = NPA_OK;
@@ -111,14 +124,16 @@ long long axis_window_sum(int L, int P, int m, int tile, bool padded) {
     return s;
 }
 
-// Key block shape: 2^lg columns x 128/2^lg rows, chosen to waste the fewest
-// key slots over all windows (ties go to the wider box: longer contiguous runs).
-int choose_kc_log2(const Geo &g) {
-    int best_lg = 7;
+// Key block shape for blocks of kb keys: 2^lg columns x kb/2^lg rows, chosen
+// to waste the fewest key slots over all windows (ties go to the wider box:
+// longer contiguous runs).
+int choose_kc_log2(const Geo &g, int kb) {
+    const int top = kb == 128 ? 7 : 6;
+    int best_lg = top;
     long long best_waste = LLONG_MAX;
     const long long exact = axis_window_sum(g.W, g.Pw, g.mw, 1, false) * axis_window_sum(g.H, g.Ph, g.mh, 1, false);
-    for (int lg = 7; lg >= 4; --lg) {
-        const int kc = 1 << lg, kr = 128 >> lg;
+    for (int lg = top; lg >= top - 3; --lg) {
+        const int kc = 1 << lg, kr = kb >> lg;
         const long long padded =
             axis_window_sum(g.W, g.Pw, g.mw, kc, true) * axis_window_sum(g.H, g.Ph, g.mh, kr, true);
         if (padded - exact < best_waste) {
@@ -202,6 +217,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     int sm_count = 0;
     npa_status st = ensure_ready(&sm_count);
     if (st != NPA_OK) return st;
+    const int nt = d == 64 ? kD64Tiles : 2;
 
     FwdParams prm;
     std::memset(&prm, 0, sizeof(prm));
@@ -218,9 +234,11 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     choose_q_tile(g.Ph, g.Pw, &prm.qc, &prm.qr);
     prm.tiles_c = (g.Pw + prm.qc - 1) / prm.qc;
     prm.tiles_r = (g.Ph + prm.qr - 1) / prm.qr;
-    prm.kc_log2 = choose_kc_log2(g);
-    prm.kr = 128 >> prm.kc_log2;
-    prm.n_qblocks = (prm.tiles_c * prm.tiles_r + 1) / 2;
+    prm.kb = nt == 3 ? 64 : 128;
+    prm.tiles_per_unit = nt;
+    prm.kc_log2 = choose_kc_log2(g, prm.kb);
+    prm.kr = prm.kb >> prm.kc_log2;
+    prm.n_qblocks = (prm.tiles_c * prm.tiles_r + nt - 1) / nt;
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     prm.wait_limit_ns = kWaitLimitNs;
 
@@ -250,7 +268,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     if (G > 0) {
         const cuuint64_t gdims[3] = {(cuuint64_t)d, (cuuint64_t)G, (cuuint64_t)BH};
         const cuuint64_t gstrides[2] = {(cuuint64_t)d * 2, (cuuint64_t)G * d * 2};
-        const cuuint32_t gbox[3] = {64, 128, 1};
+        const cuuint32_t gbox[3] = {64, (cuuint32_t)prm.kb, 1};
         if (!encode(&prm.tm_gk, gkv->k, 3, gdims, gstrides, gbox) ||
             !encode(&prm.tm_gv, gkv->v, 3, gdims, gstrides, gbox))
             return NPA_ERR_CUDA;
@@ -258,12 +276,22 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
 
     void *args[1] = {&prm};
     cudaError_t e;
-    if (d == 64)
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, false>, dim3(grid), dim3(npa::KCfg<64>::kThreads), args,
-                             npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
-    else
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, false>, dim3(grid), dim3(npa::KCfg<128>::kThreads), args,
-                             npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
+#if NPA_D64_TILES == 3
+    if (d == 64) {
+        using C = npa::KCfg<64, 3, 64>;
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, 3, 64, false>, dim3(grid), dim3(C::kThreads), args,
+                             C::kSmemBytes, (cudaStream_t)stream);
+    } else
+#endif
+    if (d == 64) {
+        using C = npa::KCfg<64, 2, 128>;
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, 2, 128, false>, dim3(grid), dim3(C::kThreads),
+                             args, C::kSmemBytes, (cudaStream_t)stream);
+    } else {
+        using C = npa::KCfg<128, 2, 128>;
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, 2, 128, false>, dim3(grid), dim3(C::kThreads),
+                             args, C::kSmemBytes, (cudaStream_t)stream);
+    }
     return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
 }
 
@@ -278,7 +306,7 @@ struct GqPlan {
 GqPlan plan_gq(int B, int heads, int H, int W, int d, int G, int sm_count) {
     GqPlan pl;
     const Geo g{H, W, H, W, 0, 0};
-    pl.kc_log2 = choose_kc_log2(g);
+    pl.kc_log2 = choose_kc_log2(g, 128);
     pl.kr = 128 >> pl.kc_log2;
     pl.n_blocks = ((W + (1 << pl.kc_log2) - 1) >> pl.kc_log2) * ((H + pl.kr - 1) / pl.kr) + (G + 127) / 128;
     const int tiles = (G + 127) / 128;
@@ -307,6 +335,8 @@ npa_status launch_gq(const void *gq, const void *k, const void *v, const void *g
     prm.Ph = H;
     prm.Pw = W;
     prm.nPh = prm.nPw = 1;
+    prm.kb = 128;
+    prm.tiles_per_unit = 2;
     prm.kc_log2 = pl.kc_log2;
     prm.kr = pl.kr;
     prm.n_qblocks = pl.n_qblocks;
@@ -333,12 +363,15 @@ npa_status launch_gq(const void *gq, const void *k, const void *v, const void *g
     const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);
     void *args[1] = {&prm};
     cudaError_t e;
-    if (d == 64)
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, true>, dim3(grid), dim3(npa::KCfg<64>::kThreads),
-                             args, npa::KCfg<64>::kSmemBytes, (cudaStream_t)stream);
-    else
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, true>, dim3(grid),
-                             dim3(npa::KCfg<128>::kThreads), args, npa::KCfg<128>::kSmemBytes, (cudaStream_t)stream);
+    if (d == 64) {
+        using C = npa::KCfg<64, 2, 128>;
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, 2, 128, true>, dim3(grid), dim3(C::kThreads),
+                             args, C::kSmemBytes, (cudaStream_t)stream);
+    } else {
+        using C = npa::KCfg<128, 2, 128>;
+        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, 2, 128, true>, dim3(grid), dim3(C::kThreads),
+                             args, C::kSmemBytes, (cudaStream_t)stream);
+    }
     if (e != cudaSuccess) return NPA_ERR_CUDA;
     if (splits > 1) {
         const int rows = prm.BH * G;

@@ -1,48 +1,52 @@
 // npa_fwd_kernel.cuh - the sm_100a forward kernel for patch-restricted
 // self-attention (NPA and PCPP share it through npa_geometry.cuh).
 //
-// One CTA per work unit: two 128-query tiles of one patch that share the
-// patch's key/value window. Three warpgroups (12 warps):
-//   warps 0-3   softmax + epilogue for query tile 0 (TMEM lanes 0..127)
-//   warps 4-7   softmax + epilogue for query tile 1
-//   warp  8     TMA producer (Q once, then K and V blocks through a ring of
-//               kStages shared-memory stages); owns the TMEM allocation
-//   warp  9     MMA issuer: d = 64, the S = Q K^T products; d = 128, all
-//   warp  10    d = 64: MMA issuer of the O += P V products
-//   warps 10-11 otherwise idle
-// The kernel is launched with 168 registers per thread; the third warpgroup
-// gives registers back (setmaxnreg.dec to kRegsCtl) and the softmax
-// warpgroups take them (setmaxnreg.inc to kRegsSoftmax):
-// 2 * 128 * kRegsSoftmax + 128 * kRegsCtl = 384 * 168, the launch's total.
+// A persistent CTA works through units of NT query tiles (128 queries each) of
+// one patch that share the patch's key/value window, streamed in blocks of KB
+// keys. Two shapes are instantiated:
+//   NT = 3, KB = 64  (image-token queries at d = 64)
+//   NT = 2, KB = 128 (d = 128, and the global-token queries)
+// Warps (NT + 1 warpgroups):
+//   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes 0..127)
+//   control warp 0     TMA producer (Q once per unit, then K and V blocks
+//                      through a ring of kStages shared-memory stages); owns
+//                      the TMEM allocation
+//   control warp 1     MMA issuer: d = 64, the S = Q K^T products; d = 128, all
+//   control warp 2     d = 64: MMA issuer of the O += P V products
+// The kernel is launched with kRegsLaunch registers per thread; the control
+// warpgroup gives registers back (setmaxnreg.dec to kRegsCtl) and the softmax
+// warpgroups take them (setmaxnreg.inc to kRegsSoftmax), NT * 128 *
+// kRegsSoftmax + 128 * kRegsCtl being the launch's total.
 //
 // Per key block j and tile q the MMA warp issues S_q = Q_q K_j^T into TMEM
-// (M=128, N=128, K=d, both operands K-major in 128-byte-swizzled shared
+// (M=128, N=KB, K=d, both operands K-major in 128-byte-swizzled shared
 // memory); the softmax warps read S_q from TMEM (one thread per query row),
 // update the running maximum and sum, and write P_q as bf16 into TMEM; the MMA
 // warp then issues O_q += P_q V_j with A = P_q read from TMEM and B = V_j
 // (MN-major, 128-byte swizzle).
 //
-// TMEM (512 columns x 128 lanes). d = 64: S0 S1 | O0 O1 | P0 P1, so P has its
-// own buffer and the MMA warp issues S_q(j+1) as soon as the softmax warps
-// have copied S_q(j) into registers: the softmax runs back to back while the
-// tensor core computes the next scores. d = 128: S0 S1 | O0 O1 with P_q in the
-// first 64 columns of S_q; the MMA warp then issues PV_q(j-1) before S_q(j),
-// and because tcgen05 operations of one thread complete in order, the commit
-// that announces S_q(j) also guarantees that PV_q(j-1) has finished. The two
-// tiles ping-pong: the tensor core works on one while the other's softmax runs.
+// TMEM (512 columns x 128 lanes). d = 64: S_0..S_{NT-1} | O_0.. | P_0.., so P
+// has its own buffer and the MMA warp issues S_q(j+1) as soon as the softmax
+// warps have copied S_q(j) into registers: the softmax runs back to back while
+// the tensor core computes the next scores. d = 128: S0 S1 | O0 O1 with P_q in
+// the first 64 columns of S_q; the MMA warp then issues PV_q(j-1) before
+// S_q(j), and because tcgen05 operations of one thread complete in order, the
+// commit that announces S_q(j) also guarantees that PV_q(j-1) has finished.
 //
-// Softmax arithmetic per block. The two softmax warpgroups take turns on the
-// exponential unit (MUFU): warpgroup q loads its scores and takes the block
-// maximum (a tree of three-input maxima) while the other group evaluates its
-// exponentials, then waits for its turn, evaluates the block's 128 x 128
-// exponentials and hands the turn back, so one group's loads, stores and
-// barrier traffic overlap the other's exponentials. p = 2^(s*log2(e)/sqrt(d)
-// - R) on the packed f32x2 FMA path and ex2.approx.f32, rounded to bf16 pairs
-// for P and summed in float32 (four packed partial sums). The reference R is
-// moved lazily: only when the block maximum exceeds it by more than
-// kRescaleLog2 (log2 units), in which case O and the row sum are rescaled by
-// 2^(R_old - R_new) before this block's P.V. P <= 2^kRescaleLog2 and the final
-// O / l is exact up to rounding.
+// Softmax arithmetic per block. At d = 64 the softmax warpgroups take turns on
+// the exponential unit (MUFU), round robin, block by block; the turn passes
+// between the warps that share a sub-partition (warp k of each group), so a
+// warp waits only for its own sub-partition's partner: warp k of group q
+// loads its scores and takes the block maximum (a tree of three-input maxima)
+// while its partner evaluates exponentials, then waits for its turn,
+// evaluates its 32 rows x KB exponentials and passes the turn on, so loads,
+// stores and barrier traffic overlap the partner's exponentials.
+// p = 2^(s*log2(e)/sqrt(d) - R) on the packed f32x2 FMA path and
+// ex2.approx.f32, rounded to bf16 pairs for P and summed in float32 (four
+// packed partial sums). The reference R is moved lazily: only when the block
+// maximum exceeds it by more than kRescaleLog2 (log2 units), in which case O
+// and the row sum are rescaled by 2^(R_old - R_new) before this block's P.V.
+// P <= 2^kRescaleLog2 and the final O / l is exact up to rounding.
 //
 // Every wait is bounded (FwdParams::wait_limit_ns). On expiry the CTA records
 // NPA_ERR_DEVICE_TIMEOUT in the device status word, stops issuing work,
@@ -62,24 +66,33 @@ __device__ unsigned int g_npa_status;  // first device-side error since last rea
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_npa_status, 0u, code); }
 
 constexpr unsigned int kErrDeviceTimeout = 5u;  // NPA_ERR_DEVICE_TIMEOUT
+
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
-template <int D>
+// Kernel shape: D = head dimension, NT = query tiles per CTA (one softmax
+// warpgroup each), KB = keys per key block.
+template <int D, int NT, int KB>
 struct KCfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static constexpr int kChunks = D / 64;              // 64-element (128-byte) column blocks
-    static constexpr int kChunkBytes = 128 * 128;       // 128 rows x 128 bytes
-    static constexpr int kTileBytes = kChunks * kChunkBytes;
-    static constexpr int kStages = (D == 64) ? 4 : 2;
-    static constexpr int kThreads = 384;
-    static constexpr uint32_t kRegsLaunch = 168;
-    static constexpr uint32_t kRegsSoftmax = 216;
-    static constexpr uint32_t kRegsCtl = 72;
-    static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl == kThreads * kRegsLaunch, "register split");
+    static_assert(NT == 2 || NT == 3, "tiles per CTA");
+    static_assert(KB == 64 || KB == 128, "keys per block");
+    static_assert(D == 64 || (NT == 2 && KB == 128), "d = 128 runs two tiles of 128-key blocks");
+    static constexpr int kChunks = D / 64;                 // 64-element (128-byte) column blocks
+    static constexpr int kQChunkBytes = 128 * 128;         // 128 query rows x 128 bytes
+    static constexpr int kQTileBytes = kChunks * kQChunkBytes;
+    static constexpr int kKVChunkBytes = KB * 128;         // KB key rows x 128 bytes
+    static constexpr int kKVTileBytes = kChunks * kKVChunkBytes;
+    static constexpr int kStages = D == 128 ? 2 : (KB == 64 ? 8 : 4);
+    static constexpr int kThreads = 128 * (NT + 1);
+    static constexpr int kCtlWarp = 4 * NT;                // first warp of the control warpgroup
+    static constexpr uint32_t kRegsLaunch = NT == 2 ? 168 : 128;
+    static constexpr uint32_t kRegsSoftmax = NT == 2 ? 216 : 144;
+    static constexpr uint32_t kRegsCtl = NT == 2 ? 72 : 80;
+    static_assert(NT * 128 * kRegsSoftmax + 128 * kRegsCtl == kThreads * kRegsLaunch, "register split");
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = 2 * kTileBytes;
-    static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+    static constexpr int kOffK = NT * kQTileBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVTileBytes;
+    static constexpr int kOffBar = kOffV + kStages * kKVTileBytes;
     // barrier indices
     static constexpr int bQFull = 0;
     static constexpr int bQEmpty = 1;                  // Q buffer free (S issuer commit after a unit)
@@ -87,25 +100,32 @@ struct KCfg {
     static constexpr int bKEmpty = bKFull + kStages;
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
-    static constexpr int bSFull = bVEmpty + kStages;   // [2] S_q written (MMA commit)
-    static constexpr int bSFree = bSFull + 2;          // [2] S_q copied to registers (128 arrivals)
-    static constexpr int bPFull = bSFree + 2;          // [2] P_q written (128 arrivals)
-    static constexpr int bPFree = bPFull + 2;          // [2] PV_q done (MMA commit)
-    static constexpr int bTurn = bPFree + 2;           // [2] exponential-phase turn of warpgroup q (4 arrivals)
-    static constexpr int bDrain = bTurn + 2;           // [2] one per MMA-issuing warp
+    static constexpr int bSFull = bVEmpty + kStages;   // [NT] S_q written (MMA commit)
+    static constexpr int bSFree = bSFull + NT;         // [NT] S_q copied to registers (128 arrivals)
+    static constexpr int bPFull = bSFree + NT;         // [NT] P_q written (128 arrivals)
+    static constexpr int bPFree = bPFull + NT;         // [NT] PV_q done (MMA commit)
+    // [NT][4] exponential-phase turn of warp k of warpgroup q (1 arrival): the
+    // turn passes between the warps that share a sub-partition's MUFU
+    static constexpr int bTurn = bPFree + NT;
+    static constexpr int bDrain = bTurn + 4 * NT;      // [2] one per MMA-issuing warp
     static constexpr int kNumBars = bDrain + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     // tensor memory columns
     static constexpr uint32_t kTmemCols = 512;
     static constexpr bool kSeparateP = (D == 64);
     // d = 64: the softmax warpgroups hand the exponential unit to each other
-    // (measured +5..7%); d = 128: the aliased-P issue order already alternates
-    // the tiles and the hand-off costs about 3%.
+    // in turn (measured +5..7% with two tiles); d = 128: the aliased-P issue
+    // order already alternates the tiles and the hand-off costs about 3%.
     static constexpr bool kUseTurn = (D == 64);
-    __device__ static constexpr uint32_t col_s(int q) { return q ? 128u : 0u; }
-    __device__ static constexpr uint32_t col_o(int q) { return 256u + (q ? uint32_t(D) : 0u); }
-    __device__ static constexpr uint32_t col_p(int q) { return kSeparateP ? (384u + (q ? 64u : 0u)) : col_s(q); }
+    __device__ static constexpr uint32_t col_s(int q) { return uint32_t(q * KB); }
+    __device__ static constexpr uint32_t col_o(int q) { return uint32_t(NT * KB + q * D); }
+    __device__ static constexpr uint32_t col_p(int q) {
+        return kSeparateP ? uint32_t(NT * KB + NT * D + q * (KB / 2)) : col_s(q);
+    }
+    static_assert(!kSeparateP || NT * KB + NT * D + NT * (KB / 2) <= 512, "tensor memory columns");
+    static_assert(kSeparateP || NT * KB + NT * D <= 512, "tensor memory columns");
 };
 
 // ---------------------------------------------------------------------------
@@ -115,37 +135,40 @@ struct KCfg {
 // Phases are counted across units: gb = key blocks processed so far by this
 // CTA (one S and one P per tile per block), uq = units processed so far.
 // ---------------------------------------------------------------------------
-template <bool GQ>
+template <int NT, bool GQ>
 __device__ __forceinline__ bool unit_has_work(const FwdParams &p, const Work &w) {
     if (GQ) return w.tile0 < p.gq_tiles && w.je > w.jb;
-    return q_tile_valid(p, w, w.tile0) || q_tile_valid(p, w, w.tile0 + 1);
+    bool any = false;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) any = any || q_tile_valid(p, w, w.tile0 + t);
+    return any;
 }
 
 // ---------------------------------------------------------------------------
-// Producer: one thread of warp 8.
+// Producer: one thread of the control warpgroup's first warp.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int NT, int KB>
 __device__ __forceinline__ void load_block(const FwdParams &p, const Work &w, int j, bool is_v, uint8_t *dst,
                                            uint64_t *bar) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     if (j < w.n_win) {
         const BlockGeom b = block_geom(p, w, j);
         const CUtensorMap *m = b.stale ? (is_v ? &p.tm_vs : &p.tm_ks) : (is_v ? &p.tm_v : &p.tm_k);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_4d(dst + c * C::kChunkBytes, m, bar, c * 64, b.col, b.row, w.bh);
+            sm100::tma_load_4d(dst + c * C::kKVChunkBytes, m, bar, c * 64, b.col, b.row, w.bh);
     } else {
-        const int g0 = (j - w.n_win) * 128;
+        const int g0 = (j - w.n_win) * KB;
         const CUtensorMap *m = is_v ? &p.tm_gv : &p.tm_gk;
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_3d(dst + c * C::kChunkBytes, m, bar, c * 64, g0, w.bh);
+            sm100::tma_load_3d(dst + c * C::kKVChunkBytes, m, bar, c * 64, g0, w.bh);
     }
 }
 
-template <int D, bool GQ>
+template <int D, int NT, int KB, bool GQ>
 __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, volatile uint32_t *abort_flag) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     const uint64_t lim = p.wait_limit_ns;
     sm100::tma_prefetch_desc(&p.tm_q);
     sm100::tma_prefetch_desc(&p.tm_k);
@@ -160,30 +183,30 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
     }
     if (GQ) sm100::tma_prefetch_desc(&p.tm_gq);
     const uint32_t q_bytes = GQ ? uint32_t(C::kChunks * 128 * 128) : uint32_t(C::kChunks * p.qc * p.qr * 128);
-    int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q pairs issued
+    int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q tile groups issued
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
         const Work w = decode<GQ>(p, unit);
-        if (!unit_has_work<GQ>(p, w)) continue;
+        if (!unit_has_work<NT, GQ>(p, w)) continue;
         // the previous unit's last S products must be done with the Q buffer
         if (uq > 0 && !sm100::mbar_wait(&bars[C::bQEmpty], (uq - 1) & 1, lim)) {
             ok = false;
             break;
         }
-        sm100::mbar_arrive_expect_tx(&bars[C::bQFull], 2 * q_bytes);
+        sm100::mbar_arrive_expect_tx(&bars[C::bQFull], NT * q_bytes);
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < NT; ++t) {
             if (GQ) {
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_3d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_gq,
+                    sm100::tma_load_3d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_gq,
                                        &bars[C::bQFull], c * 64, (w.tile0 + t) * 128, w.bh);
             } else {
                 int row0, col0;
                 q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_4d(smem + C::kOffQ + t * C::kTileBytes + c * C::kChunkBytes, &p.tm_q,
+                    sm100::tma_load_4d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_q,
                                        &bars[C::bQFull], c * 64, col0, row0, w.bh);
             }
         }
@@ -198,15 +221,15 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
                 ok = false;
                 break;
             }
-            sm100::mbar_arrive_expect_tx(&bars[C::bKFull + s], C::kTileBytes);
-            load_block<D>(p, w, j, false, smem + C::kOffK + s * C::kTileBytes, &bars[C::bKFull + s]);
+            sm100::mbar_arrive_expect_tx(&bars[C::bKFull + s], C::kKVTileBytes);
+            load_block<D, NT, KB>(p, w, j, false, smem + C::kOffK + s * C::kKVTileBytes, &bars[C::bKFull + s]);
             ++nk;
             if (use > 0 && !sm100::mbar_wait(&bars[C::bVEmpty + s], (use - 1) & 1, lim)) {
                 ok = false;
                 break;
             }
-            sm100::mbar_arrive_expect_tx(&bars[C::bVFull + s], C::kTileBytes);
-            load_block<D>(p, w, j, true, smem + C::kOffV + s * C::kTileBytes, &bars[C::bVFull + s]);
+            sm100::mbar_arrive_expect_tx(&bars[C::bVFull + s], C::kKVTileBytes);
+            load_block<D, NT, KB>(p, w, j, true, smem + C::kOffV + s * C::kKVTileBytes, &bars[C::bVFull + s]);
             ++nv;
         }
     }
@@ -230,43 +253,45 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
 // through K (16 elements = 32 bytes inside a 128-byte swizzle atom, or the
 // next 64-column block) or through the keys of V only adds a constant to the
 // start-address field.
-template <int D>
+template <int D, int NT, int KB>
 __device__ __forceinline__ void issue_s(uint32_t tmem, int q, uint64_t qdesc, uint64_t kdesc) {
-    using C = KCfg<D>;
-    constexpr uint32_t kIdS = sm100::idesc_bf16_f32(128, 128, false, false);  // S = Q K^T
+    using C = KCfg<D, NT, KB>;
+    constexpr uint32_t kIdS = sm100::idesc_bf16_f32(128, KB, false, false);  // S = Q K^T
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t off = uint64_t(((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4);
-        sm100::mma_ss(tmem + C::col_s(q), qdesc + off, kdesc + off, kIdS, kk > 0 ? 1u : 0u);
+        const uint64_t qoff = uint64_t(((kk >> 2) * C::kQChunkBytes + (kk & 3) * 32) >> 4);
+        const uint64_t koff = uint64_t(((kk >> 2) * C::kKVChunkBytes + (kk & 3) * 32) >> 4);
+        sm100::mma_ss(tmem + C::col_s(q), qdesc + qoff, kdesc + koff, kIdS, kk > 0 ? 1u : 0u);
     }
 }
 
-template <int D>
+template <int D, int NT, int KB>
 __device__ __forceinline__ void issue_pv(uint32_t tmem, int q, uint64_t vdesc, bool accumulate) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     constexpr uint32_t kIdO = sm100::idesc_bf16_f32(128, D, false, true);  // O += P V, V MN-major
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
+    for (int kk = 0; kk < KB / 16; ++kk)
         sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p(q) + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), kIdO,
                       (accumulate || kk > 0) ? 1u : 0u);
 }
 
 struct OperandDescs {
-    uint64_t q0, q1, k0, v0;  // Q tiles, K and V stage 0
-    uint64_t stage;           // descriptor increment from one stage to the next
+    uint64_t q0, k0, v0;  // Q tile 0, K and V stage 0
+    uint64_t qtile;       // descriptor increment from one Q tile to the next
+    uint64_t stage;       // descriptor increment from one K/V stage to the next
 };
 
-template <int D>
+template <int D, int NT, int KB>
 __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     OperandDescs d;
     // K-major operands: SBO = 8 rows x 128 bytes. V (MN-major): LBO = next
     // 64-column block, SBO = next 8 keys.
     d.q0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffQ), 16, 1024);
-    d.q1 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffQ + C::kTileBytes), 16, 1024);
     d.k0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffK), 16, 1024);
-    d.v0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffV), C::kChunkBytes, 1024);
-    d.stage = uint64_t(C::kTileBytes >> 4);
+    d.v0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffV), C::kKVChunkBytes, 1024);
+    d.qtile = uint64_t(C::kQTileBytes >> 4);
+    d.stage = uint64_t(C::kKVTileBytes >> 4);
     return d;
 }
 
@@ -275,17 +300,17 @@ __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
 // independently. This one issues S_0(j), S_1(j) as soon as the softmax warps
 // hold S(j-1) in registers; the first S of a unit also overlaps the previous
 // unit's last P.V products and epilogue.
-template <int D, bool GQ>
+template <int D, int NT, int KB, bool GQ>
 __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                           volatile uint32_t *abort_flag) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     const uint64_t lim = p.wait_limit_ns;
-    const OperandDescs dd = make_descs<D>(smem);
+    const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0, uq = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
         const Work w = decode<GQ>(p, unit);
-        if (!unit_has_work<GQ>(p, w)) continue;
+        if (!unit_has_work<NT, GQ>(p, w)) continue;
         ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
         for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
@@ -295,11 +320,11 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
             }
             const int s = gb % C::kStages;
             ok = sm100::mbar_wait(&bars[C::bKFull + s], (gb / C::kStages) & 1, lim);
-            for (int q = 0; ok && q < 2; ++q) {
+            for (int q = 0; ok && q < NT; ++q) {
                 if (gb > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (gb - 1) & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + s * dd.stage);
+                issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + s * dd.stage);
                 sm100::tc_commit(&bars[C::bSFull + q]);
             }
             if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
@@ -315,17 +340,17 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
 }
 
 // d = 64: the P.V products, O_q(j) += P_q(j) V(j) as each P_q(j) arrives.
-template <int D, bool GQ>
+template <int D, int NT, int KB, bool GQ>
 __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                            volatile uint32_t *abort_flag) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     const uint64_t lim = p.wait_limit_ns;
-    const OperandDescs dd = make_descs<D>(smem);
+    const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
         const Work w = decode<GQ>(p, unit);
-        if (!unit_has_work<GQ>(p, w)) continue;
+        if (!unit_has_work<NT, GQ>(p, w)) continue;
         for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
             if (*abort_flag) {
                 ok = false;
@@ -333,11 +358,11 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
             }
             const int s = gb % C::kStages;
             ok = sm100::mbar_wait(&bars[C::bVFull + s], (gb / C::kStages) & 1, lim);
-            for (int q = 0; ok && q < 2; ++q) {
+            for (int q = 0; ok && q < NT; ++q) {
                 ok = sm100::mbar_wait(&bars[C::bPFull + q], gb & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                issue_pv<D>(tmem, q, dd.v0 + s * dd.stage, j > w.jb);
+                issue_pv<D, NT, KB>(tmem, q, dd.v0 + s * dd.stage, j > w.jb);
                 sm100::tc_commit(&bars[C::bPFree + q]);
             }
             if (ok) sm100::tc_commit(&bars[C::bVEmpty + s]);
@@ -353,17 +378,17 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
 
 // d = 128 (P aliases S): one warp issues everything, PV_q(j-1) before S_q(j)
 // for each tile, so that the completion of S_q(j) also implies PV_q(j-1).
-template <int D, bool GQ>
+template <int D, int NT, int KB, bool GQ>
 __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
                         volatile uint32_t *abort_flag) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     const uint64_t lim = p.wait_limit_ns;
-    const OperandDescs dd = make_descs<D>(smem);
+    const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0, uq = 0;  // gb: global index of block j = 0 of the current unit
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
         const Work w = decode<GQ>(p, unit);
-        if (!unit_has_work<GQ>(p, w)) continue;
+        if (!unit_has_work<NT, GQ>(p, w)) continue;
         const int n = w.je - w.jb;  // blocks of this unit, counted from its first
         ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
@@ -383,16 +408,16 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
                 if (!ok) break;
             }
             sm100::tc_fence_after();
-            for (int q = 0; q < 2; ++q) {
+            for (int q = 0; q < NT; ++q) {
                 if (j > 0) {
                     ok = sm100::mbar_wait(&bars[C::bPFull + q], (g - 1) & 1, lim);
                     if (!ok) break;
                     sm100::tc_fence_after();
-                    issue_pv<D>(tmem, q, dd.v0 + ((g - 1) % C::kStages) * dd.stage, j > 1);
+                    issue_pv<D, NT, KB>(tmem, q, dd.v0 + ((g - 1) % C::kStages) * dd.stage, j > 1);
                     sm100::tc_commit(&bars[C::bPFree + q]);
                 }
                 if (j < n) {
-                    issue_s<D>(tmem, q, q ? dd.q1 : dd.q0, dd.k0 + (g % C::kStages) * dd.stage);
+                    issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + (g % C::kStages) * dd.stage);
                     sm100::tc_commit(&bars[C::bSFull + q]);
                 }
             }
@@ -420,14 +445,18 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64
 }
 
 // Row maximum of 128 scores: eight independent chains of three-input maxima.
-__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+// Maximum of a row's KB scores: eight interleaved chains of three-input maxima.
+template <int KB>
+__device__ __forceinline__ float row_max(const float (&s)[KB]) {
+    constexpr int kLen = KB / 8;  // elements per chain: k, k + 8, k + 16, ...
     float mk[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         float m = sm100::max3(s[k], s[k + 8], s[k + 16]);
 #pragma unroll
-        for (int t = 3; t < 15; t += 2) m = sm100::max3(m, s[k + 8 * t], s[k + 8 * t + 8]);
-        mk[k] = fmaxf(m, s[k + 120]);
+        for (int t = 3; t + 1 < kLen; t += 2) m = sm100::max3(m, s[k + 8 * t], s[k + 8 * t + 8]);
+        if (kLen % 2 == 0) m = fmaxf(m, s[k + 8 * (kLen - 1)]);
+        mk[k] = m;
     }
     return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
 }
@@ -465,14 +494,15 @@ __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float &p0, float &p1) 
     p1 = x1 < -125.f ? 0.f : __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-// p = 2^(s*c - ref) for 128 scores: packed bf16 pairs into pk, float32 sum returned.
-__device__ __forceinline__ float exp_block(const float (&s)[128], float c, float ref, uint32_t (&pk)[64]) {
+// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum returned.
+template <int KB>
+__device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2]) {
     const float neg = (ref == -INFINITY) ? 0.f : -ref;
     const uint64_t c2 = sm100::pack_f32x2(c, c);
     const uint64_t m2 = sm100::pack_f32x2(neg, neg);
     uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
+    for (int i = 0; i < KB / 2; ++i) {
         const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
         float p0, p1;
         if ((i & 7) < NPA_EXP_EMU8) {
@@ -494,14 +524,15 @@ __device__ __forceinline__ float exp_block(const float (&s)[128], float c, float
     return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
-template <int D, bool GQ>
+template <int D, int NT, int KB, bool GQ>
 __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
                             int q) {
-    using C = KCfg<D>;
+    using C = KCfg<D, NT, KB>;
     const uint64_t lim = p.wait_limit_ns;
     const int row = threadIdx.x & 127;
     const bool lane0 = (threadIdx.x & 31) == 0;
-    const uint32_t lane_off = uint32_t((threadIdx.x >> 5) & 3) * 32u << 16;
+    const int warp_in_group = (threadIdx.x >> 5) & 3;
+    const uint32_t lane_off = uint32_t(warp_in_group) * 32u << 16;
     const uint32_t tS = tmem + lane_off + C::col_s(q);
     const uint32_t tO = tmem + lane_off + C::col_o(q);
     const uint32_t tP = tmem + lane_off + C::col_p(q);
@@ -511,7 +542,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
     const Work w = decode<GQ>(p, unit);
-    if (!unit_has_work<GQ>(p, w)) continue;
+    if (!unit_has_work<NT, GQ>(p, w)) continue;
     // window block coordinates, advanced without divisions: column block,
     // first row of the current band, end of the band's row segment
     int btc = 0, brow = w.seg[0], bend = w.seg[1];
@@ -529,12 +560,15 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             break;
         }
         sm100::tc_fence_after();
-        float s[128];
+        float s[KB];
         {
-            uint32_t sr[128];
-            sm100::tmem_ld128(tS, sr);
+            uint32_t sr[KB];
+            if constexpr (KB == 128)
+                sm100::tmem_ld128(tS, sr);
+            else
+                sm100::tmem_ld64(tS, sr);
 #pragma unroll
-            for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+            for (int i = 0; i < KB; ++i) s[i] = __uint_as_float(sr[i]);
         }
         if (C::kSeparateP) {
             // S_q may be overwritten by the next block's scores
@@ -548,7 +582,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             const int vr = bend - brow;
             if (vc < kc || vr < p.kr) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
+                for (int i = 0; i < KB; ++i)
                     if ((i & (kc - 1)) >= vc || (i >> p.kc_log2) >= vr) s[i] = -INFINITY;
             }
             if (++btc == w.wtc) {
@@ -560,30 +594,32 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
                 }
             }
         } else {
-            const int vg = p.G - (j - w.n_win) * 128;
-            if (vg < 128) {
+            const int vg = p.G - (j - w.n_win) * KB;
+            if (vg < KB) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i)
+                for (int i = 0; i < KB; ++i)
                     if (i >= vg) s[i] = -INFINITY;
             }
         }
         // block maximum and the reference for this block's P (lazy: the
         // reference moves only when the maximum grows by more than kRescaleLog2)
-        const float bm = row_max128(s) * sl2;
+        const float bm = row_max<KB>(s) * sl2;
         if (bm > R + kRescaleLog2) R = bm;
-        // wait for this warpgroup's turn on the exponential unit
-        if (C::kUseTurn && (q == 1 || gb > 0) &&
-            !warp_wait(&bars[C::bTurn + q], (q == 0 ? gb - 1 : gb) & 1, lim)) {
+        // wait for this warpgroup's turn on the exponential unit (the turn
+        // goes round the warpgroups in order, block by block)
+        if (C::kUseTurn && (q > 0 || gb > 0) &&
+            !warp_wait(&bars[C::bTurn + 4 * q + warp_in_group], (q == 0 ? gb - 1 : gb) & 1, lim)) {
             ok = false;
             break;
         }
-        uint32_t pk[64];
-        const float blk_sum = exp_block(s, sl2, R, pk);
-        // the turn passes only once the whole block is issued (handing it over
-        // at 5/8, 3/4 or 7/8 of the block measured 16% slower)
+        uint32_t pk[KB / 2];
+        const float blk_sum = exp_block<KB>(s, sl2, R, pk);
+        // pass the turn to the next warpgroup's warp on this sub-partition
+        // once the whole block is issued (handing it over at 3/4 or 7/8 of
+        // the block measured 16-17% slower)
         if (C::kUseTurn) {
             __syncwarp();
-            if (lane0) sm100::mbar_arrive(&bars[C::bTurn + (q ^ 1)]);
+            if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
         }
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
         if (C::kSeparateP && j > w.jb) {
@@ -605,7 +641,10 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
         }
         l = l * alpha + blk_sum;
-        sm100::tmem_st64(tP, pk);
+        if constexpr (KB == 128)
+            sm100::tmem_st64(tP, pk);
+        else
+            sm100::tmem_st32(tP, pk);
         sm100::tc_fence_before();
         sm100::mbar_arrive(&bars[C::bPFull + q]);
         R_prev = R;
@@ -676,9 +715,9 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int D, bool GQ>
-__global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
-    using C = KCfg<D>;
+template <int D, int NT, int KB, bool GQ>
+__global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
+    using C = KCfg<D, NT, KB>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = sm100::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -696,19 +735,19 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
             sm100::mbar_init(&bars[C::bVFull + s], 1);
             sm100::mbar_init(&bars[C::bVEmpty + s], 1);
         }
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < NT; ++q) {
             sm100::mbar_init(&bars[C::bSFull + q], 1);
             sm100::mbar_init(&bars[C::bSFree + q], 128);
             sm100::mbar_init(&bars[C::bPFull + q], 128);
             sm100::mbar_init(&bars[C::bPFree + q], 1);
-            sm100::mbar_init(&bars[C::bTurn + q], 4);
+            for (int k = 0; k < 4; ++k) sm100::mbar_init(&bars[C::bTurn + 4 * q + k], 1);
         }
         sm100::mbar_init(&bars[C::bDrain], 1);
         sm100::mbar_init(&bars[C::bDrain + 1], 1);
         misc[1] = 0;
         sm100::fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == C::kCtlWarp) {
         sm100::tmem_alloc(&misc[0], C::kTmemCols);
         sm100::tmem_relinquish();
     }
@@ -718,26 +757,27 @@ __global__ void __launch_bounds__(384, 1) npa_fwd_kernel(const __grid_constant__
     const uint32_t tmem = misc[0];
     volatile uint32_t *abort_flag = &misc[1];
 
-    if (warp >= 8) {
+    if (warp >= C::kCtlWarp) {
         sm100::setmaxnreg_dec<C::kRegsCtl>();
+        const int role = warp - C::kCtlWarp;
         if ((threadIdx.x & 31) == 0) {
-            if (warp == 8) run_producer<D, GQ>(p, smem, bars, abort_flag);
+            if (role == 0) run_producer<D, NT, KB, GQ>(p, smem, bars, abort_flag);
             if (C::kSeparateP) {
-                if (warp == 9) run_mma_s<D, GQ>(p, smem, bars, tmem, abort_flag);
-                if (warp == 10) run_mma_pv<D, GQ>(p, smem, bars, tmem, abort_flag);
-            } else if (warp == 9) {
-                run_mma<D, GQ>(p, smem, bars, tmem, abort_flag);
+                if (role == 1) run_mma_s<D, NT, KB, GQ>(p, smem, bars, tmem, abort_flag);
+                if (role == 2) run_mma_pv<D, NT, KB, GQ>(p, smem, bars, tmem, abort_flag);
+            } else if (role == 1) {
+                run_mma<D, NT, KB, GQ>(p, smem, bars, tmem, abort_flag);
             }
         }
     } else {
         sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D, GQ>(p, bars, tmem, abort_flag, warp >> 2);
+        run_softmax<D, NT, KB, GQ>(p, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();
     __syncthreads();
     sm100::tc_fence_after();
-    if (warp == 8) {
+    if (warp == C::kCtlWarp) {
         __syncwarp();
         sm100::tmem_dealloc(tmem, C::kTmemCols);
     }

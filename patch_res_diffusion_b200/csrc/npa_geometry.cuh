@@ -10,12 +10,13 @@
 //     window of strip i is rows [i*s - r, (i+1)*s + r) clipped, all columns:
 //     the strip plus the r adjacent rows of each neighbouring strip.
 //
-// Work unit = (batch*head, patch, pair of 128-row query tiles); a persistent
-// CTA walks the units blockIdx.x, blockIdx.x + gridDim.x, ... A query tile is
-// a box of qr patch rows x qc patch columns (qr*qc <= 128); a key/value block
-// is a box of kr rows x kc columns (kr*kc = 128) inside the window, followed
-// by ceil(G/128) blocks of global tokens. Every quantity is recomputed from
-// the unit index with integer arithmetic; there are no index tables.
+// Work unit = (batch*head, patch, group of tiles_per_unit 128-row query
+// tiles); a persistent CTA walks the units blockIdx.x, blockIdx.x + gridDim.x,
+// ... A query tile is a box of qr patch rows x qc patch columns (qr*qc <=
+// 128); a key/value block is a box of kr rows x kc columns (kr*kc = kb, 64 or
+// 128 keys) inside the window, followed by ceil(G/kb) blocks of global
+// tokens. Every quantity is recomputed from the unit index with integer
+// arithmetic; the only table is the host-built patch order.
 #pragma once
 
 #include <cstdint>
@@ -32,7 +33,7 @@ struct FwdParams {
     CUtensorMap tm_q;   // 4D {d, W, H, B*heads}, box {64, qc, qr, 1}, 128B swizzle
     CUtensorMap tm_k;   // 4D, box {64, kc, kr, 1}
     CUtensorMap tm_v;   // 4D, box {64, kc, kr, 1}
-    CUtensorMap tm_gk;  // 3D {d, G, B*heads}, box {64, 128, 1} (unused when G == 0)
+    CUtensorMap tm_gk;  // 3D {d, G, B*heads}, box {64, kb, 1} (unused when G == 0)
     CUtensorMap tm_gv;
     CUtensorMap tm_ks;  // previous step's K / V for the borrowed rows (two_source only)
     CUtensorMap tm_vs;
@@ -42,15 +43,17 @@ struct FwdParams {
     int Ph, Pw, mh, mw;
     int nPh, nPw;                    // patches along rows / columns
     int qc, qr, tiles_c, tiles_r;    // query tile box and tiles per patch
+    int kb;                          // keys per key block (64 or 128)
     int kc_log2, kr;                 // key block box: (1 << kc_log2) columns x kr rows
-    int n_qblocks;                   // query-tile pairs per patch
+    int tiles_per_unit;              // query tiles per work unit (2 or 3)
+    int n_qblocks;                   // query-tile groups per patch
     float scale_log2;                // log2(e) / sqrt(d)
     unsigned long long wait_limit_ns;
     int BH;                          // batch * heads
     int n_units;                     // work units in execution order
     int two_source;                  // 1: rows outside the patch come from tm_ks / tm_vs
     int patch_begin, patch_count;    // patches computed (natural order when n_perm == 0)
-    int n_splits;                    // global-token queries: key-range splits per query tile pair
+    int n_splits;                    // global-token queries: key-range splits per query tile group
     int gq_tiles;                    // global-token queries: ceil(G / 128)
     float *o_part;                   // splits > 1: [n_splits][B*heads][G][d] unnormalised O
     float *ml;                       // splits > 1: [n_splits][B*heads][G][2] reference max, row sum
@@ -70,7 +73,7 @@ struct Work {
     int wr0, wr1, wc0, wc1;   // clipped window
     int seg[4];               // row segment boundaries (see above)
     int nb0, nb01;            // key blocks of segment 0, of segments 0 and 1
-    int tile0;                // first query tile (of two) within the patch
+    int tile0;                // first query tile of the unit's group within the patch
     int wtc;                  // window blocks along the columns
     int n_win, n_blocks;      // window blocks, window + global blocks
     int jb, je;               // the unit's key blocks [jb, je) (a key-range split)
@@ -145,7 +148,7 @@ inline void order_patches(FwdParams &prm) {
 
 // Work units are ordered by cost class (patches with the same number of key
 // blocks, largest first), then batch*head, then patch within the class, then
-// query-tile pair. The cheapest units come last, and the units running at the
+// query-tile group. The cheapest units come last, and the units running at the
 // same time are the neighbouring patches of a few heads, whose overlapping
 // key/value windows are then read from L2 rather than DRAM (one launch of
 // B2 h10 256x256 patch 64 margin 32 read 0.84 GB from DRAM in this order,
@@ -177,7 +180,7 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     w.wr1 = imin_(p.H, w.pr1 + p.mh);
     w.wc0 = imax_(0, w.pc0 - p.mw);
     w.wc1 = imin_(p.W, w.pc1 + p.mw);
-    w.tile0 = 2 * qb;
+    w.tile0 = p.tiles_per_unit * qb;
     const int kc = 1 << p.kc_log2;
     w.wtc = cdiv_(w.wc1 - w.wc0, kc);
     if (p.two_source) {
@@ -192,7 +195,7 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     w.nb0 = w.wtc * cdiv_(w.seg[1] - w.seg[0], p.kr);
     w.nb01 = w.nb0 + w.wtc * cdiv_(w.seg[2] - w.seg[1], p.kr);
     w.n_win = w.nb01 + w.wtc * cdiv_(w.seg[3] - w.seg[2], p.kr);
-    w.n_blocks = w.n_win + cdiv_(p.G, 128);
+    w.n_blocks = w.n_win + cdiv_(p.G, p.kb);
     w.jb = 0;
     w.je = w.n_blocks;
     w.split = 0;
@@ -200,7 +203,7 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
 }
 
 // Global-token queries (the text-query half of joint attention): a unit is
-// (batch*head, key-range split, pair of 128-token query tiles); the window is
+// (batch*head, key-range split, group of 128-token query tiles); the window is
 // the whole grid followed by the global tokens, and split s covers key
 // blocks [s*n/S, (s+1)*n/S).
 __host__ __device__ inline Work decode_work_gq(const FwdParams &p, int unit) {
@@ -217,11 +220,11 @@ __host__ __device__ inline Work decode_work_gq(const FwdParams &p, int unit) {
     w.wc1 = p.W;
     w.seg[0] = w.seg[1] = 0;
     w.seg[2] = w.seg[3] = p.H;
-    w.tile0 = 2 * qb;
+    w.tile0 = p.tiles_per_unit * qb;
     w.wtc = cdiv_(p.W, 1 << p.kc_log2);
     w.nb0 = 0;
     w.nb01 = w.n_win = w.wtc * cdiv_(p.H, p.kr);
-    w.n_blocks = w.n_win + cdiv_(p.G, 128);
+    w.n_blocks = w.n_win + cdiv_(p.G, p.kb);
     w.jb = (int)((long long)w.split * w.n_blocks / p.n_splits);
     w.je = (int)((long long)(w.split + 1) * w.n_blocks / p.n_splits);
     return w;

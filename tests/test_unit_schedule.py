@@ -29,19 +29,22 @@ def run(exe, *args):
     return {"units": int(f[2]), "ordered": int(f[4]), "classes": int(f[6]), "wave_heads": int(f[8])}
 
 
-# BH, H, W, Ph, Pw, mh, mw, kc_log2, n_qblocks, patch_begin, patch_count
+# BH, H, W, Ph, Pw, mh, mw, kb, kc_log2, tiles_per_unit, n_qblocks, patch_begin, patch_count
 CASES = {
-    "npa_sdxl_4096": (20, 256, 256, 64, 64, 32, 32, 5, 16, 0, -1),
-    "npa_flux_4096": (24, 256, 256, 64, 64, 32, 32, 5, 16, 0, -1),
-    "npa_sdxl_2048": (20, 128, 128, 64, 64, 32, 32, 5, 16, 0, -1),
-    "ragged": (3, 40, 37, 16, 16, 5, 5, 4, 1, 0, -1),
-    "ragged_small_patches": (2, 100, 100, 9, 9, 3, 3, 3, 1, 0, -1),
-    "pcpp_4x32": (20, 128, 128, 32, 128, 8, 0, 7, 16, 0, -1),
-    "pcpp_strip_range": (4, 64, 64, 8, 64, 3, 0, 6, 2, 3, 4),
-    "npa_patch_range": (4, 64, 64, 16, 16, 4, 4, 4, 1, 3, 7),
-    "unordered": (2, 61, 59, 3, 4, 1, 2, 3, 1, 0, -1),        # 315 patches: natural order
-    "fifteen_classes": (2, 300, 300, 20, 20, 60, 60, 3, 1, 0, -1),
-    "too_many_classes": (2, 300, 300, 20, 20, 100, 100, 3, 1, 0, -1),  # ordered, no class table
+    "npa_sdxl_4096": (20, 256, 256, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
+    "npa_sdxl_4096_triples": (20, 256, 256, 64, 64, 32, 32, 64, 5, 3, 11, 0, -1),  # NPA_D64_TILES=3
+    "npa_flux_4096": (24, 256, 256, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
+    "npa_sdxl_2048": (20, 128, 128, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
+    "ragged": (3, 40, 37, 16, 16, 5, 5, 64, 4, 3, 1, 0, -1),
+    "ragged_small_patches": (2, 100, 100, 9, 9, 3, 3, 128, 3, 2, 1, 0, -1),
+    "pcpp_4x32": (20, 128, 128, 32, 128, 10, 0, 128, 7, 2, 16, 0, -1),
+    "pcpp_8x16": (20, 128, 128, 16, 128, 13, 0, 128, 7, 2, 8, 0, -1),
+    "pcpp_8x16_triples": (20, 128, 128, 16, 128, 13, 0, 64, 6, 3, 6, 0, -1),
+    "pcpp_strip_range": (4, 64, 64, 8, 64, 3, 0, 128, 6, 2, 2, 3, 4),
+    "npa_patch_range": (4, 64, 64, 16, 16, 4, 4, 64, 4, 3, 1, 3, 7),
+    "unordered": (2, 61, 59, 3, 4, 1, 2, 128, 3, 2, 1, 0, -1),        # 315 patches: natural order
+    "fifteen_classes": (2, 300, 300, 20, 20, 60, 60, 128, 3, 2, 1, 0, -1),
+    "too_many_classes": (2, 300, 300, 20, 20, 100, 100, 128, 3, 2, 1, 0, -1),  # ordered, no class table
 }
 
 
@@ -50,17 +53,20 @@ def test_every_unit_once_cheapest_last(checker, name):
     r = run(checker, *CASES[name], 148)
     a = CASES[name]
     n_patches = ((a[1] + a[3] - 1) // a[3]) * ((a[2] + a[4] - 1) // a[4])
-    count = n_patches - a[9] if a[10] < 0 else a[10]
-    assert r["units"] == a[0] * count * a[8]
+    count = n_patches - a[11] if a[12] < 0 else a[12]
+    assert r["units"] == a[0] * count * a[10]
 
 
 def test_concurrent_units_share_heads(checker):
     """SDXL 4096^2 (B2 h10, 4x4 patches of 64, margin 32): the windows fall in
-    3 cost classes, and the first 148 units (one per SM) cover only 3 of the
-    20 batch*heads, so their overlapping windows are shared in L2."""
+    3 cost classes, and the first 148 units (one per SM) cover only 3 to 5 of
+    the 20 batch*heads, so their overlapping windows are shared in L2."""
     r = run(checker, *CASES["npa_sdxl_4096"], 148)
     assert r["classes"] == 3
     assert r["wave_heads"] <= 3
+    r = run(checker, *CASES["npa_sdxl_4096_triples"], 148)
+    assert r["classes"] == 3
+    assert r["wave_heads"] <= 5
 
 
 def test_fallbacks(checker):

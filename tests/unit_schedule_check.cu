@@ -1,7 +1,7 @@
 // Host-only check of the persistent kernel's work-unit schedule: for one
 // geometry given on the command line it decodes every unit index and checks
 // that each (batch*head, patch, query-tile pair) of the patch range occurs
-// exactly once, that unit costs never increase along the order when an
+// (a group of tiles_per_unit query tiles) exactly once, that unit costs never increase along the order when an
 // order was built (at most kMaxPatchOrder patches), and prints the number of
 // ordered patches, the number of cost classes and the batch*head values the
 // first `wave` units touch. Built and run by test_unit_schedule.py.
@@ -14,12 +14,12 @@
 #include "../patch_res_diffusion_b200/csrc/npa_geometry.cuh"
 
 int main(int argc, char **argv) {
-    if (argc != 13) {
-        std::fprintf(stderr, "usage: BH H W Ph Pw mh mw kc_log2 n_qblocks patch_begin patch_count wave\n");
+    if (argc != 15) {
+        std::fprintf(stderr, "usage: BH H W Ph Pw mh mw kb kc_log2 tiles_per_unit n_qblocks patch_begin patch_count wave\n");
         return 2;
     }
-    int a[12];
-    for (int i = 0; i < 12; ++i) a[i] = std::atoi(argv[i + 1]);
+    int a[14];
+    for (int i = 0; i < 14; ++i) a[i] = std::atoi(argv[i + 1]);
     npa::FwdParams p;
     std::memset(&p, 0, sizeof(p));
     p.BH = a[0];
@@ -29,14 +29,16 @@ int main(int argc, char **argv) {
     p.Pw = a[4];
     p.mh = a[5];
     p.mw = a[6];
-    p.kc_log2 = a[7];
-    p.kr = 128 >> p.kc_log2;
-    p.n_qblocks = a[8];
+    p.kb = a[7];
+    p.kc_log2 = a[8];
+    p.kr = p.kb >> p.kc_log2;
+    p.tiles_per_unit = a[9];
+    p.n_qblocks = a[10];
     p.nPh = (p.H + p.Ph - 1) / p.Ph;
     p.nPw = (p.W + p.Pw - 1) / p.Pw;
-    p.patch_begin = a[9];
-    p.patch_count = a[10] < 0 ? p.nPh * p.nPw - p.patch_begin : a[10];
-    const int wave = a[11];
+    p.patch_begin = a[11];
+    p.patch_count = a[12] < 0 ? p.nPh * p.nPw - p.patch_begin : a[12];
+    const int wave = a[13];
     p.n_units = p.BH * p.patch_count * p.n_qblocks;
     npa::order_patches(p);
     const int n_patches = p.nPh * p.nPw;
@@ -46,8 +48,8 @@ int main(int argc, char **argv) {
     for (int u = 0; u < p.n_units; ++u) {
         const npa::Work w = npa::decode_work(p, u);
         const int patch = (w.pr0 / p.Ph) * p.nPw + w.pc0 / p.Pw;
-        const int qb = w.tile0 / 2;
-        if (w.bh < 0 || w.bh >= p.BH || patch < p.patch_begin || patch >= p.patch_begin + p.patch_count ||
+        const int qb = w.tile0 / p.tiles_per_unit;
+        if (w.tile0 % p.tiles_per_unit != 0 || w.bh < 0 || w.bh >= p.BH || patch < p.patch_begin || patch >= p.patch_begin + p.patch_count ||
             qb < 0 || qb >= p.n_qblocks) {
             std::printf("FAIL unit %d decodes outside the range (bh %d patch %d pair %d)\n", u, w.bh, patch, qb);
             return 1;
