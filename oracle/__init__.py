@@ -36,6 +36,7 @@ __all__ = [
     "lib", "npa_key_set", "pcpp_key_set", "pcpp_neighbor_rows", "npa_attention",
     "pcpp_attention", "pcpp_attention_stale", "pair_count", "num_threads", "dense_mask",
     "dense_attention", "dense_pcpp_stale", "global_query_attention", "bf16_to_f64",
+    "multidiffusion_attention", "md_window_keys", "md_window_count", "md_pair_count",
 ]
 
 _LIB = None
@@ -67,6 +68,15 @@ def lib() -> ctypes.CDLL:
         L.oracle_global_query_attention.argtypes = [u16p] * 5 + [ctypes.c_void_p] + [ctypes.c_int] * 6 + [
             ctypes.c_void_p, ctypes.c_long]
         L.oracle_global_query_attention.restype = ctypes.c_int
+        L.oracle_multidiffusion_attention.argtypes = common + [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                               ctypes.c_void_p, ctypes.c_long]
+        L.oracle_multidiffusion_attention.restype = ctypes.c_int
+        L.oracle_md_window_keys.argtypes = [ctypes.c_int] * 6 + [i32p]
+        L.oracle_md_window_keys.restype = ctypes.c_int
+        L.oracle_md_window_count.argtypes = [ctypes.c_int] * 5
+        L.oracle_md_window_count.restype = ctypes.c_int
+        L.oracle_md_pair_count.argtypes = [ctypes.c_int] * 5
+        L.oracle_md_pair_count.restype = ctypes.c_longlong
         L.oracle_pair_count.argtypes = [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
         L.oracle_pair_count.restype = ctypes.c_longlong
         L.oracle_num_threads.argtypes = []
@@ -157,6 +167,41 @@ def pcpp_attention(q, k, v, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None,
     """PCPP attention in float64. ``queries``: optional (n, 3) array of (b, h, t)."""
     return _call(lib().oracle_pcpp_attention, (n_strips, float(p)), q, k, v, gk, gv, B, heads, H,
                  W, d, G, queries)
+
+
+def multidiffusion_attention(q, k, v, *, B, heads, H, W, d, patch, margin, gk=None, gv=None, G=0,
+                             queries: Optional[Sequence] = None) -> np.ndarray:
+    """Overlapping-window (MultiDiffusion-style) attention in float64: every
+    NPA window attends within itself; a token's output is the mean over the
+    windows that contain it. ``queries``: optional (n, 3) array of (b, h, t)."""
+    return _call(lib().oracle_multidiffusion_attention, (patch, margin), q, k, v, gk, gv, B, heads, H, W, d,
+                 G, queries)
+
+
+def md_window_keys(H: int, W: int, patch: int, margin: int, pi: int, pj: int) -> np.ndarray:
+    """Token ids of window (pi, pj), ascending."""
+    out = np.empty(H * W, dtype=np.int32)
+    n = lib().oracle_md_window_keys(H, W, patch, margin, pi, pj,
+                                    out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    if n < 0:
+        raise ValueError("bad window arguments")
+    return out[:n].copy()
+
+
+def md_window_count(H: int, W: int, patch: int, margin: int, t: int) -> int:
+    """Number of windows containing token t."""
+    n = lib().oracle_md_window_count(H, W, patch, margin, t)
+    if n < 0:
+        raise ValueError("bad arguments")
+    return int(n)
+
+
+def md_pair_count(H: int, W: int, patch: int, margin: int, G: int = 0) -> int:
+    """(query, key) pairs of one (b, h) under overlapping-window attention."""
+    n = lib().oracle_md_pair_count(H, W, patch, margin, G)
+    if n < 0:
+        raise ValueError("bad arguments")
+    return int(n)
 
 
 def pcpp_attention_stale(q, k, v, ks, vs, *, B, heads, H, W, d, n_strips, p, gk=None, gv=None, G=0,

@@ -325,6 +325,130 @@ int oracle_global_query_attention(const uint16_t *gq, const uint16_t *k, const u
     return status;
 }
 
+/* ------------------------------------------------------------------ */
+/* MultiDiffusion-style overlapping-window attention (comparator).      */
+/* ------------------------------------------------------------------ */
+/* ScaleDiff summary, "Approach" and "Problem": MultiDiffusion covers the
+ * latent with overlapping patches, processes each patch on its own and
+ * averages the overlaps; NPA instead keeps the query patches disjoint and
+ * lets each attend to an overlapping neighbourhood. Reading taken here, at
+ * the level of one attention layer and with the NPA windows as the
+ * overlapping patches: window (pi, pj) is NPA patch (pi, pj) grown by m and
+ * clipped; inside each window every token attends to every token of that
+ * window (plus the G global tokens); a token's output is the mean, over the
+ * windows that contain it, of its attention output in each. */
+
+/* Window (pi, pj) as row range [r0, r1) x column range [c0, c1). */
+static void md_window(int H, int W, int P, int m, int pi, int pj, int *r0, int *r1, int *c0, int *c1) {
+    *r0 = imax(0, pi * P - m);
+    *r1 = imin(H, (pi + 1) * P + m);
+    *c0 = imax(0, pj * P - m);
+    *c1 = imin(W, (pj + 1) * P + m);
+}
+
+/* Tokens of window (pi, pj), ascending. Returns the count or -1. */
+int oracle_md_window_keys(int H, int W, int P, int m, int pi, int pj, int32_t *out) {
+    if (H < 1 || W < 1 || P < 1 || m < 0) return -1;
+    int nph = (H + P - 1) / P, npw = (W + P - 1) / P;
+    if (pi < 0 || pi >= nph || pj < 0 || pj >= npw) return -1;
+    int r0, r1, c0, c1, n = 0;
+    md_window(H, W, P, m, pi, pj, &r0, &r1, &c0, &c1);
+    for (int r = r0; r < r1; ++r)
+        for (int c = c0; c < c1; ++c) out[n++] = r * W + c;
+    return n;
+}
+
+/* Number of windows that contain token t, by testing every window. */
+int oracle_md_window_count(int H, int W, int P, int m, int t) {
+    if (H < 1 || W < 1 || P < 1 || m < 0 || t < 0 || t >= H * W) return -1;
+    int r = t / W, c = t % W, n = 0;
+    for (int pi = 0; pi < (H + P - 1) / P; ++pi)
+        for (int pj = 0; pj < (W + P - 1) / P; ++pj) {
+            int r0, r1, c0, c1;
+            md_window(H, W, P, m, pi, pj, &r0, &r1, &c0, &c1);
+            n += (r >= r0 && r < r1 && c >= c0 && c < c1);
+        }
+    return n;
+}
+
+/* (query, key) pairs of one (b, h): sum over windows of |W| (|W| + G). */
+long long oracle_md_pair_count(int H, int W, int P, int m, int G) {
+    if (H < 1 || W < 1 || P < 1 || m < 0 || G < 0) return -1;
+    long long total = 0;
+    for (int pi = 0; pi < (H + P - 1) / P; ++pi)
+        for (int pj = 0; pj < (W + P - 1) / P; ++pj) {
+            int r0, r1, c0, c1;
+            md_window(H, W, P, m, pi, pj, &r0, &r1, &c0, &c1);
+            long long n = (long long)(r1 - r0) * (c1 - c0);
+            total += n * (n + G);
+        }
+    return total;
+}
+
+/* Overlapping-window attention for a list of (b, h, t) queries (NULL: all,
+ * out is then [B, heads, H*W, d]). */
+int oracle_multidiffusion_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                    const uint16_t *gk, const uint16_t *gv, double *out,
+                                    int B, int heads, int H, int W, int d, int P, int m, int G,
+                                    const int32_t *queries, long n_queries) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || P < 1 || m < 0 || G < 0) return ORACLE_BAD_ARG;
+    if (G > 0 && (!gk || !gv)) return ORACLE_BAD_ARG;
+    const long N = (long)H * W;
+    const long total = queries ? n_queries : (long)B * heads * N;
+    const int nph = (H + P - 1) / P, npw = (W + P - 1) / P;
+    int status = ORACLE_OK;
+#pragma omp parallel
+    {
+        int32_t *keys = (int32_t *)malloc(sizeof(int32_t) * (size_t)N);
+        double *z = (double *)malloc(sizeof(double) * (size_t)(N + G));
+        double *o_w = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!keys || !z || !o_w) {
+#pragma omp critical
+            status = ORACLE_NOMEM;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long i = 0; i < total; ++i) {
+                long bb, hh, t;
+                if (queries) {
+                    bb = queries[3 * i]; hh = queries[3 * i + 1]; t = queries[3 * i + 2];
+                    if (bb < 0 || bb >= B || hh < 0 || hh >= heads || t < 0 || t >= N) {
+#pragma omp critical
+                        status = ORACLE_BAD_ARG;
+                        continue;
+                    }
+                } else {
+                    t = i % N; hh = (i / N) % heads; bb = i / (N * heads);
+                }
+                size_t bh = (size_t)bb * heads + hh;
+                double *o = out + (size_t)i * d;
+                for (int c = 0; c < d; ++c) o[c] = 0.0;
+                int count = 0, r = (int)(t / W), col = (int)(t % W);
+                for (int pi = 0; pi < nph; ++pi)
+                    for (int pj = 0; pj < npw; ++pj) {
+                        int r0, r1, c0, c1;
+                        md_window(H, W, P, m, pi, pj, &r0, &r1, &c0, &c1);
+                        if (r < r0 || r >= r1 || col < c0 || col >= c1) continue;
+                        int n_img = oracle_md_window_keys(H, W, P, m, pi, pj, keys);
+                        int rc = attend_one(q + (bh * N + t) * d, k + bh * N * d, v + bh * N * d, NULL, NULL, NULL,
+                                            G ? gk + bh * (size_t)G * d : NULL, G ? gv + bh * (size_t)G * d : NULL,
+                                            G, d, keys, n_img, z, o_w);
+                        if (rc != ORACLE_OK) {
+#pragma omp critical
+                            status = rc;
+                        }
+                        for (int c = 0; c < d; ++c) o[c] += o_w[c];
+                        ++count;
+                    }
+                for (int c = 0; c < d; ++c) o[c] /= (double)count;
+            }
+        }
+        free(keys);
+        free(z);
+        free(o_w);
+    }
+    return status;
+}
+
 /* Number of (query, key) pairs, summed over all queries of one (b, h),
  * counting image keys and global keys. Brute force over every token. */
 long long oracle_pair_count(int geom, int H, int W, int a, int b, double p, int G) {
