@@ -31,7 +31,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import PRESETS, Workload, make_inputs  # noqa: E402
+from workloads import COMPARATORS, PRESETS, Workload, make_inputs, preset  # noqa: E402
 
 DEFAULT_WORKLOAD = "npa_sdxl_4096"
 L2_BYTES = 126 * 1024 * 1024
@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(PRESETS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(PRESETS) + sorted(COMPARATORS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -56,8 +56,10 @@ def parse():
 
 def describe(w: Workload) -> dict:
     cfg = {"workload": w.name, "B": w.B, "heads": w.heads, "grid": f"{w.H}x{w.W}", "d": w.d}
-    if w.geometry == "npa":
-        cfg.update({"geometry": "npa", "patch": w.patch, "margin": w.margin})
+    if w.geometry in ("npa", "md"):
+        cfg.update({"geometry": w.geometry, "patch": w.patch, "margin": w.margin})
+        if w.geometry == "md":
+            cfg["comparator"] = "overlapping NPA windows, each attending within itself, outputs averaged"
     else:
         cfg.update({"geometry": "pcpp", "n_strips": w.n_strips, "p": w.p})
     cfg["global_tokens"] = w.G
@@ -102,6 +104,8 @@ def useful_flops(w: Workload) -> float:
     import patch_res_diffusion_b200 as npa
     if w.geometry == "npa":
         return npa.npa_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
+    if w.geometry == "md":
+        return npa.npa_multidiffusion_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
     return npa.pcpp_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, w.G)
 
 
@@ -115,15 +119,22 @@ def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
     import oracle
     rng = np.random.default_rng(123)
     N = w.H * w.W
-    geom = dict(patch=w.patch, margin=w.margin) if w.geometry == "npa" else dict(n_strips=w.n_strips, p=w.p)
-    fn = oracle.npa_attention if w.geometry == "npa" else oracle.pcpp_attention
-    key_count = (lambda t: len(oracle.npa_key_set(w.H, w.W, w.patch, w.margin, t))) if w.geometry == "npa" \
-        else (lambda t: len(oracle.pcpp_key_set(w.H, w.W, w.n_strips, w.p, t)))
+    geom = dict(patch=w.patch, margin=w.margin) if w.geometry in ("npa", "md") else \
+        dict(n_strips=w.n_strips, p=w.p)
+    fn = {"npa": oracle.npa_attention, "md": oracle.multidiffusion_attention}.get(w.geometry,
+                                                                                  oracle.pcpp_attention)
+    if w.geometry == "npa":
+        key_count = lambda t: len(oracle.npa_key_set(w.H, w.W, w.patch, w.margin, t))
+    elif w.geometry == "md":
+        key_count = lambda t: md_query_pairs(w, t) - w.G * md_cover(w, t)
+    else:
+        key_count = lambda t: len(oracle.pcpp_key_set(w.H, w.W, w.n_strips, w.p, t))
     n, total_q, total_pairs, total_t = 64, 0, 0, 0.0
     while total_t < seconds:
         qs = np.stack([rng.integers(w.B, size=n), rng.integers(w.heads, size=n), rng.integers(N, size=n)],
                       axis=1).astype(np.int32)
-        pairs = sum(key_count(int(t)) + w.G for t in qs[:, 2])
+        pairs = sum(key_count(int(t)) + w.G * (md_cover(w, int(t)) if w.geometry == "md" else 1)
+                    for t in qs[:, 2])
         t0 = time.perf_counter()
         fn(inp["q"], inp["k"], inp["v"], gk=inp.get("gk"), gv=inp.get("gv"), G=w.G, B=w.B, heads=w.heads,
            H=w.H, W=w.W, d=w.d, queries=qs, **geom)
@@ -141,6 +152,28 @@ def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
         "sample": f"{total_q} uniformly drawn (b, h, query) rows of {w.name}, float64, {total_t:.1f} s",
         "seconds": total_t,
     }
+
+
+def _md_axis(L: int, P: int, m: int, x: int):
+    """Extents of the windows containing coordinate x along one axis."""
+    out = []
+    for i in range((L + P - 1) // P):
+        lo, hi = max(0, i * P - m), min(L, (i + 1) * P + m)
+        if lo <= x < hi:
+            out.append(hi - lo)
+    return out
+
+
+def md_cover(w: Workload, t: int) -> int:
+    """Windows containing token t (overlapping-window comparator)."""
+    return len(_md_axis(w.H, w.patch, w.margin, t // w.W)) * len(_md_axis(w.W, w.patch, w.margin, t % w.W))
+
+
+def md_query_pairs(w: Workload, t: int) -> int:
+    """(query, key) pairs the comparator evaluates for token t: its window's
+    keys (plus the global keys) in every window containing it."""
+    rows, cols = _md_axis(w.H, w.patch, w.margin, t // w.W), _md_axis(w.W, w.patch, w.margin, t % w.W)
+    return sum(rows) * sum(cols) + w.G * len(rows) * len(cols)
 
 
 def run_reference(args, w: Workload, rank: int) -> None:
@@ -180,6 +213,8 @@ def run_reference(args, w: Workload, rank: int) -> None:
 
 def useful_flops_host(w: Workload) -> float:
     import oracle
+    if w.geometry == "md":
+        return 4.0 * w.d * w.B * w.heads * oracle.md_pair_count(w.H, w.W, w.patch, w.margin, w.G)
     pairs = oracle.pair_count(w.geometry, w.H, w.W, patch=w.patch, margin=w.margin, n_strips=w.n_strips,
                               p=w.p, G=w.G)
     return 4.0 * w.d * w.B * w.heads * pairs
@@ -270,9 +305,16 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     needs_flush = bytes_io < 2 * L2_BYTES
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if needs_flush else None
 
+    md_bytes = npa.npa_multidiffusion_workspace_size(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin) \
+        if w.geometry == "md" else 0
+    md_ws = [torch.empty(md_bytes, dtype=torch.uint8, device=dev) for _ in range(2)] if md_bytes else None
+
     def call():
         if w.geometry == "npa":
             npa.npa_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, gk, gv, w.G, stream)
+        elif w.geometry == "md":
+            npa.npa_multidiffusion_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin,
+                                                 md_ws[0], md_bytes, gk, gv, w.G, stream)
         else:
             npa.pcpp_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, gk, gv, w.G, stream)
 
@@ -359,6 +401,9 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
                 if w.geometry == "npa":
                     npa.npa_attention_fwd(bq, bk, bv, bo, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, bgk, bgv,
                                           w.G, stream)
+                elif w.geometry == "md":
+                    npa.npa_multidiffusion_attention_fwd(bq, bk, bv, bo, w.B, w.heads, w.H, w.W, w.d, w.patch,
+                                                         w.margin, md_ws[b], md_bytes, bgk, bgv, w.G, stream)
                 else:
                     npa.pcpp_attention_fwd(bq, bk, bv, bo, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, bgk,
                                            bgv, w.G, stream)
@@ -401,7 +446,8 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "peak_kind": f"{pk_kind} bf16 burst",
         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
         "frac_of_datasheet_dense": achieved / DATASHEET_BF16_DENSE_TFLOPS,
-        "kernel": KERNEL_NAME, "useful_flops_per_launch": flops,
+        "kernel": KERNEL_NAME if w.geometry != "md" else
+        KERNEL_NAME + " + md_combine_kernel (timed together: one call)", "useful_flops_per_launch": flops,
         "avg_launch_ms": avg_kernel_ms,
         "hbm_min_bytes_per_launch": bytes_io,
     }
@@ -431,7 +477,7 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if w.geometry == "md" else 1),
         "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
     }
     print(json.dumps(line), flush=True)
@@ -439,7 +485,7 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
 
 def main():
     args = parse()
-    w = PRESETS[args.workload]
+    w = preset(args.workload)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

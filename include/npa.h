@@ -153,6 +153,37 @@ npa_status npa_global_query_attention_fwd_noalloc(const void *gq, const void *k,
                                                   const void *gv, void *go, int B, int heads, int H, int W,
                                                   int d, int G, npa_stream_t stream);
 
+/* Overlapping-window attention, the comparator NPA is measured against
+ * (ScaleDiff summary, "Problem" and "Approach": MultiDiffusion processes
+ * overlapping patches and averages them, which inflates the attention cost;
+ * NPA keeps the query patches disjoint). The overlapping patches are the NPA
+ * windows: window (pi, pj) is patch (pi, pj) grown by `margin` and clipped to
+ * the grid; every token of a window attends to every token of that window
+ * (plus the global tokens), and a token's output is the mean, over the windows
+ * that contain it, of its attention output in each. This reading of the
+ * comparison at the level of one attention layer is the library's; the pages
+ * compare whole pipelines.
+ * Runs the attention kernel over all windows, writing each window's
+ * normalised float32 output to `workspace` (caller-owned device memory,
+ * 16-byte aligned, at least npa_multidiffusion_workspace_size() bytes, not
+ * overlapping any other buffer), then a second kernel on the same stream that
+ * averages them into o. At most 256 patches along each axis
+ * (NPA_ERR_UNSUPPORTED beyond). A NULL or short workspace gives
+ * NPA_ERR_INVALID_ARG. Other arguments and errors as for npa_attention_fwd. */
+npa_status npa_multidiffusion_attention_fwd(const void *q, const void *k, const void *v, void *o, int B, int heads,
+                                            int H, int W, int d, int patch, int margin,
+                                            const npa_global_kv *global_kv, void *workspace,
+                                            size_t workspace_bytes, npa_stream_t stream);
+
+/* Workspace bytes of npa_multidiffusion_attention_fwd: 4 * d * B * heads *
+ * (sum of window heights) * (sum of window widths); 0 for invalid arguments. */
+size_t npa_multidiffusion_workspace_size(int B, int heads, int H, int W, int d, int patch, int margin);
+
+/* Useful floating-point work of one npa_multidiffusion_attention_fwd call:
+ * 4 * d * B * heads * sum over windows of |window| * (|window| + G). Negative
+ * for invalid arguments. */
+double npa_multidiffusion_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G);
+
 /* Workspace bytes npa_global_query_attention_fwd uses for its full split
  * count on the current device (0: no split needed, or invalid arguments). */
 size_t npa_global_query_workspace_size(int B, int heads, int H, int W, int d, int G);

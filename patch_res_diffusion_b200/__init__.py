@@ -12,6 +12,10 @@ a call fails, an exception is raised.
 * ``pcpp_attention_fwd`` - partially conditioned attention (PCPP review, "What
   carries the argument"): row strips attending to themselves plus the nearest
   ceil(p * rows) rows of each adjacent strip.
+* ``npa_multidiffusion_attention_fwd`` - the overlapping-window comparator
+  (ScaleDiff summary, "Approach": MultiDiffusion averages overlapping
+  patches): each NPA window attends within itself and a token's output is the
+  mean over the windows that contain it.
 """
 from __future__ import annotations
 
@@ -26,7 +30,8 @@ __all__ = [
     "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string", "npa_attention",
     "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "npa_global_query_attention_fwd",
     "npa_global_query_workspace_size", "npa_global_query_attention_fwd_noalloc", "global_query_attention",
-    "EXPORTED_SYMBOLS",
+    "npa_multidiffusion_attention_fwd", "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops",
+    "multidiffusion_attention", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
@@ -42,7 +47,8 @@ EXPORTED_SYMBOLS = (
     "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_attention_fwd_stale", "pcpp_neighbor_rows", "npa_useful_flops",
     "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
     "npa_global_query_attention_fwd", "npa_global_query_workspace_size",
-    "npa_global_query_attention_fwd_noalloc",
+    "npa_global_query_attention_fwd_noalloc", "npa_multidiffusion_attention_fwd",
+    "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops",
 )
 
 
@@ -78,6 +84,13 @@ def lib() -> ctypes.CDLL:
         L.npa_global_query_attention_fwd.restype = i
         L.npa_global_query_attention_fwd_noalloc.argtypes = [vp] * 6 + [i] * 6 + [vp]
         L.npa_global_query_attention_fwd_noalloc.restype = i
+        L.npa_multidiffusion_attention_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, gkv, vp,
+                                                       ctypes.c_size_t, vp]
+        L.npa_multidiffusion_attention_fwd.restype = i
+        L.npa_multidiffusion_workspace_size.argtypes = [i] * 7
+        L.npa_multidiffusion_workspace_size.restype = ctypes.c_size_t
+        L.npa_multidiffusion_useful_flops.argtypes = [i] * 8
+        L.npa_multidiffusion_useful_flops.restype = d
         L.npa_global_query_workspace_size.argtypes = [i] * 6
         L.npa_global_query_workspace_size.restype = ctypes.c_size_t
         L.pcpp_neighbor_rows.argtypes = [i, d]
@@ -174,6 +187,25 @@ def npa_global_query_attention_fwd_noalloc(gq, k, v, gk, gv, go, B: int, heads: 
            "npa_global_query_attention_fwd_noalloc")
 
 
+def npa_multidiffusion_attention_fwd(q, k, v, o, B: int, heads: int, H: int, W: int, d: int, patch: int,
+                                     margin: int, workspace, workspace_bytes: int, global_k=None, global_v=None,
+                                     n_global: int = 0, stream=None) -> None:
+    """C ``npa_multidiffusion_attention_fwd``: overlapping-window attention;
+    ``workspace`` holds npa_multidiffusion_workspace_size() bytes."""
+    _check(lib().npa_multidiffusion_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), B, heads, H, W, d, patch,
+                                                  margin, _gkv(global_k, global_v, n_global), _ptr(workspace),
+                                                  int(workspace_bytes), _stream(stream)),
+           "npa_multidiffusion_attention_fwd")
+
+
+def npa_multidiffusion_workspace_size(B, heads, H, W, d, patch, margin) -> int:
+    return int(lib().npa_multidiffusion_workspace_size(B, heads, H, W, d, patch, margin))
+
+
+def npa_multidiffusion_useful_flops(B, heads, H, W, d, patch, margin, G=0) -> float:
+    return float(lib().npa_multidiffusion_useful_flops(B, heads, H, W, d, patch, margin, G))
+
+
 def npa_global_query_workspace_size(B, heads, H, W, d, G) -> int:
     return int(lib().npa_global_query_workspace_size(B, heads, H, W, d, G))
 
@@ -265,4 +297,21 @@ def global_query_attention(gq, k, v, gk, gv, H: int, W: int, out=None, split: bo
         if nbytes:
             ws = torch.empty(nbytes, dtype=torch.uint8, device=gq.device)
     npa_global_query_attention_fwd(gq, k, v, gk, gv, out, B, heads, H, W, d, G, ws, nbytes, stream)
+    return out
+
+
+def multidiffusion_attention(q, k, v, H: int, W: int, patch: int, margin: int, global_k=None, global_v=None,
+                             out=None, workspace=None, stream=None):
+    """Overlapping-window attention on torch bf16 CUDA tensors [B, heads,
+    H*W, d]; allocates the float32 window workspace unless one is given."""
+    import torch
+    B, heads, d = _shape(q, H, W)
+    if out is None:
+        out = q.new_empty(q.shape)
+    nbytes = npa_multidiffusion_workspace_size(B, heads, H, W, d, patch, margin)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    G = 0 if global_k is None else int(global_k.shape[2])
+    npa_multidiffusion_attention_fwd(q, k, v, out, B, heads, H, W, d, patch, margin, workspace,
+                                     workspace.numel() * workspace.element_size(), global_k, global_v, G, stream)
     return out

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -82,6 +83,8 @@ npa_status ensure_ready(int *sm_count = nullptr) {
 #endif
                    !set_smem(npa::npa_fwd_kernel<64, 2, 128, false>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<128, 2, 128, false>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
+                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, false, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
+                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, false, true>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<64, 2, 128, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<128, 2, 128, true>, npa::KCfg<128, 2, 128>::kSmemBytes)) {
             return NPA_ERR_CUDA;
@@ -167,6 +170,37 @@ void choose_q_tile(int Ph, int Pw, int *qc_out, int *qr_out) {
     *qr_out = br;
 }
 
+// Overlapping-window mode: the query tile box (qc columns x qr rows, qc*qr <=
+// 128) that needs the fewest tiles over all windows; windows form a grid, so
+// the count is (sum over column windows of ceil(width/qc)) x (sum over row
+// windows of ceil(height/qr)). tiles_c / tiles_r cover the largest window.
+void choose_q_tile_md(const Geo &g, int *qc_out, int *qr_out, int *tiles_c, int *tiles_r) {
+    const int nph = (g.H + g.Ph - 1) / g.Ph, npw = (g.W + g.Pw - 1) / g.Pw;
+    long long best = LLONG_MAX;
+    for (int qc = 128; qc >= 8; qc /= 2) {
+        const int qr = 128 / qc;
+        long long sc = 0, sr = 0;
+        int mc = 0, mr = 0;
+        for (int j = 0; j < npw; ++j) {
+            const int ww = std::min(g.W, (j + 1) * g.Pw + g.mw) - std::max(0, j * g.Pw - g.mw);
+            sc += (ww + qc - 1) / qc;
+            mc = std::max(mc, (ww + qc - 1) / qc);
+        }
+        for (int i = 0; i < nph; ++i) {
+            const int wh = std::min(g.H, (i + 1) * g.Ph + g.mh) - std::max(0, i * g.Ph - g.mh);
+            sr += (wh + qr - 1) / qr;
+            mr = std::max(mr, (wh + qr - 1) / qr);
+        }
+        if (sc * sr < best) {
+            best = sc * sr;
+            *qc_out = qc;
+            *qr_out = qr;
+            *tiles_c = mc;
+            *tiles_r = mr;
+        }
+    }
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
@@ -213,11 +247,11 @@ npa_status validate_common(const void *q, const void *k, const void *v, void *o,
 // patches computed, in natural numbering; patch_count < 0 means all.
 npa_status launch(const void *q, const void *k, const void *v, const void *ks, const void *vs, void *o, int B,
                   int heads, int d, const Geo &g, int G, const npa_global_kv *gkv, int patch_begin, int patch_count,
-                  npa_stream_t stream) {
+                  npa_stream_t stream, float *md_part = nullptr) {
     int sm_count = 0;
     npa_status st = ensure_ready(&sm_count);
     if (st != NPA_OK) return st;
-    const int nt = d == 64 ? kD64Tiles : 2;
+    const int nt = (d == 64 && !md_part) ? kD64Tiles : 2;
 
     FwdParams prm;
     std::memset(&prm, 0, sizeof(prm));
@@ -231,9 +265,18 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     prm.mw = g.mw;
     prm.nPh = (g.H + g.Ph - 1) / g.Ph;
     prm.nPw = (g.W + g.Pw - 1) / g.Pw;
-    choose_q_tile(g.Ph, g.Pw, &prm.qc, &prm.qr);
-    prm.tiles_c = (g.Pw + prm.qc - 1) / prm.qc;
-    prm.tiles_r = (g.Ph + prm.qr - 1) / prm.qr;
+    if (md_part) {
+        if (prm.nPh > npa::kMaxMdAxis || prm.nPw > npa::kMaxMdAxis) return NPA_ERR_UNSUPPORTED;
+        choose_q_tile_md(g, &prm.qc, &prm.qr, &prm.tiles_c, &prm.tiles_r);
+        prm.md = 1;
+        prm.md_part = md_part;
+        prm.md_rows = npa::md_axis_offset(g.H, g.Ph, g.mh, prm.nPh);
+        prm.md_tw = npa::md_axis_offset(g.W, g.Pw, g.mw, prm.nPw);
+    } else {
+        choose_q_tile(g.Ph, g.Pw, &prm.qc, &prm.qr);
+        prm.tiles_c = (g.Pw + prm.qc - 1) / prm.qc;
+        prm.tiles_r = (g.Ph + prm.qr - 1) / prm.qr;
+    }
     prm.kb = nt == 3 ? 64 : 128;
     prm.tiles_per_unit = nt;
     prm.kc_log2 = choose_kc_log2(g, prm.kb);
@@ -276,23 +319,63 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
 
     void *args[1] = {&prm};
     cudaError_t e;
+    const void *kernel;
+    unsigned threads, smem;
+    if (d == 64 && md_part) {
+        kernel = (const void *)npa::npa_fwd_kernel<64, 2, 128, false, true>;
+        threads = npa::KCfg<64, 2, 128>::kThreads;
+        smem = npa::KCfg<64, 2, 128>::kSmemBytes;
+    } else if (d == 128 && md_part) {
+        kernel = (const void *)npa::npa_fwd_kernel<128, 2, 128, false, true>;
+        threads = npa::KCfg<128, 2, 128>::kThreads;
+        smem = npa::KCfg<128, 2, 128>::kSmemBytes;
 #if NPA_D64_TILES == 3
-    if (d == 64) {
-        using C = npa::KCfg<64, 3, 64>;
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, 3, 64, false>, dim3(grid), dim3(C::kThreads), args,
-                             C::kSmemBytes, (cudaStream_t)stream);
-    } else
+    } else if (d == 64) {
+        kernel = (const void *)npa::npa_fwd_kernel<64, 3, 64, false>;
+        threads = npa::KCfg<64, 3, 64>::kThreads;
+        smem = npa::KCfg<64, 3, 64>::kSmemBytes;
 #endif
-    if (d == 64) {
-        using C = npa::KCfg<64, 2, 128>;
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<64, 2, 128, false>, dim3(grid), dim3(C::kThreads),
-                             args, C::kSmemBytes, (cudaStream_t)stream);
+    } else if (d == 64) {
+        kernel = (const void *)npa::npa_fwd_kernel<64, 2, 128, false>;
+        threads = npa::KCfg<64, 2, 128>::kThreads;
+        smem = npa::KCfg<64, 2, 128>::kSmemBytes;
     } else {
-        using C = npa::KCfg<128, 2, 128>;
-        e = cudaLaunchKernel((const void *)npa::npa_fwd_kernel<128, 2, 128, false>, dim3(grid), dim3(C::kThreads),
-                             args, C::kSmemBytes, (cudaStream_t)stream);
+        kernel = (const void *)npa::npa_fwd_kernel<128, 2, 128, false>;
+        threads = npa::KCfg<128, 2, 128>::kThreads;
+        smem = npa::KCfg<128, 2, 128>::kSmemBytes;
     }
-    return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
+    e = cudaLaunchKernel(kernel, dim3(grid), dim3(threads), args, smem, (cudaStream_t)stream);
+    if (e != cudaSuccess) return NPA_ERR_CUDA;
+    if (md_part) {
+        npa::MdCombineParams cp;
+        std::memset(&cp, 0, sizeof(cp));
+        cp.part = md_part;
+        cp.o = static_cast<__nv_bfloat16 *>(o);
+        cp.H = g.H;
+        cp.W = g.W;
+        cp.Ph = g.Ph;
+        cp.Pw = g.Pw;
+        cp.mh = g.mh;
+        cp.mw = g.mw;
+        cp.nPh = prm.nPh;
+        cp.nPw = prm.nPw;
+        cp.BH = BH;
+        cp.md_rows = prm.md_rows;
+        cp.md_tw = prm.md_tw;
+        for (int i = 0; i < prm.nPh; ++i) cp.rh[i] = npa::md_axis_offset(g.H, g.Ph, g.mh, i);
+        for (int j = 0; j < prm.nPw; ++j) cp.cw[j] = npa::md_axis_offset(g.W, g.Pw, g.mw, j);
+        void *cargs[1] = {&cp};
+        const long long tokens = (long long)BH * g.H * g.W;
+        const dim3 cgrid((unsigned)((tokens + 7) / 8));
+        if (d == 64)
+            e = cudaLaunchKernel((const void *)npa::md_combine_kernel<64>, cgrid, dim3(256), cargs, 0,
+                                 (cudaStream_t)stream);
+        else
+            e = cudaLaunchKernel((const void *)npa::md_combine_kernel<128>, cgrid, dim3(256), cargs, 0,
+                                 (cudaStream_t)stream);
+        if (e != cudaSuccess) return NPA_ERR_CUDA;
+    }
+    return NPA_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -429,6 +512,13 @@ int neighbor_rows(int s, double p) {
     return r;
 }
 
+// Overlapping-window mode: bytes of float32 window partials.
+size_t md_workspace_bytes(int B, int heads, int H, int W, int d, int patch, int margin) {
+    const long long rows = npa::md_axis_offset(H, patch, margin, (H + patch - 1) / patch);
+    const long long cols = npa::md_axis_offset(W, patch, margin, (W + patch - 1) / patch);
+    return (size_t)B * heads * rows * cols * d * sizeof(float);
+}
+
 double useful_flops(int B, int heads, int d, const Geo &g, int G) {
     const double pairs = (double)axis_pair_sum(g.H, g.Ph, g.mh) * (double)axis_pair_sum(g.W, g.Pw, g.mw) +
                          (double)g.H * g.W * G;
@@ -544,6 +634,51 @@ npa_status npa_global_query_attention_fwd_noalloc(const void *gq, const void *k,
     float *o_part = splits > 1 ? static_cast<float *>(base) : nullptr;
     float *ml = splits > 1 ? o_part + (size_t)splits * B * heads * G * d : nullptr;
     return launch_gq(gq, k, v, gk, gv, go, B, heads, H, W, d, G, o_part, ml, splits, sm_count, stream);
+}
+
+size_t npa_multidiffusion_workspace_size(int B, int heads, int H, int W, int d, int patch, int margin) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || patch < 1 || margin < 0 || (d != 64 && d != 128)) return 0;
+    return md_workspace_bytes(B, heads, H, W, d, patch, margin);
+}
+
+npa_status npa_multidiffusion_attention_fwd(const void *q, const void *k, const void *v, void *o, int B, int heads,
+                                            int H, int W, int d, int patch, int margin,
+                                            const npa_global_kv *global_kv, void *workspace,
+                                            size_t workspace_bytes, npa_stream_t stream) {
+    int G = 0;
+    npa_status st = validate_common(q, k, v, o, B, heads, H, W, d, global_kv, &G);
+    if (st != NPA_OK) return st;
+    if (patch < 1 || margin < 0 || !workspace) return NPA_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return NPA_ERR_MISALIGNED;
+    const long long nph = (H + patch - 1) / patch, npw = (W + patch - 1) / patch;
+    if (nph > npa::kMaxMdAxis || npw > npa::kMaxMdAxis) return NPA_ERR_UNSUPPORTED;
+    const size_t need = md_workspace_bytes(B, heads, H, W, d, patch, margin);
+    if (workspace_bytes < need) return NPA_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)B * heads * H * W * d * 2, gbytes = (size_t)B * heads * G * d * 2;
+    if (overlaps(workspace, need, q, bytes) || overlaps(workspace, need, k, bytes) ||
+        overlaps(workspace, need, v, bytes) || overlaps(workspace, need, o, bytes))
+        return NPA_ERR_INVALID_ARG;
+    if (G && (overlaps(workspace, need, global_kv->k, gbytes) || overlaps(workspace, need, global_kv->v, gbytes)))
+        return NPA_ERR_INVALID_ARG;
+    const Geo g{H, W, patch, patch, margin, margin};
+    return launch(q, k, v, nullptr, nullptr, o, B, heads, d, g, G, global_kv, 0, -1, stream,
+                  static_cast<float *>(workspace));
+}
+
+double npa_multidiffusion_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G) {
+    if (B < 1 || heads < 1 || H < 1 || W < 1 || d < 1 || patch < 1 || margin < 0 || G < 0) return -1.0;
+    double s1r = 0, s2r = 0, s1c = 0, s2c = 0;
+    for (int i = 0; i < (H + patch - 1) / patch; ++i) {
+        const double w = std::min(H, (i + 1) * patch + margin) - std::max(0, i * patch - margin);
+        s1r += w;
+        s2r += w * w;
+    }
+    for (int j = 0; j < (W + patch - 1) / patch; ++j) {
+        const double w = std::min(W, (j + 1) * patch + margin) - std::max(0, j * patch - margin);
+        s1c += w;
+        s2c += w * w;
+    }
+    return 4.0 * d * (double)B * heads * (s2r * s2c + G * s1r * s1c);
 }
 
 int pcpp_neighbor_rows(int strip_rows, double p) { return neighbor_rows(strip_rows, p); }

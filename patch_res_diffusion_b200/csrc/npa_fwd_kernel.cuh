@@ -524,7 +524,7 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
     return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
-template <int D, int NT, int KB, bool GQ>
+template <int D, int NT, int KB, bool GQ, bool MD>
 __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
                             int q) {
     using C = KCfg<D, NT, KB>;
@@ -687,6 +687,29 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         const int grow = row0 + rr, gcol = col0 + cc;
         valid = t < p.tiles_c * p.tiles_r && row < p.qc * p.qr && grow < w.pr1 && gcol < w.pc1;
         out_row = (size_t)w.bh * p.H * p.W + (size_t)grow * p.W + gcol;
+        if constexpr (MD) {
+            // overlapping windows: this window's normalised output, float32,
+            // at the token's place in the window's block of the partials
+            int bh_unused;
+            const int patch = unit_patch(p, unit, &bh_unused);
+            const int rh = md_axis_offset(p.H, p.Ph, p.mh, patch / p.nPw);
+            const int cw = md_axis_offset(p.W, p.Pw, p.mw, patch % p.nPw);
+            const size_t prow = ((size_t)w.bh * p.md_rows + (rh + grow - w.wr0)) * p.md_tw + (cw + gcol - w.wc0);
+            float4 *part = reinterpret_cast<float4 *>(p.md_part + prow * D);
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                sm100::tmem_ld32(tO + c * 32, o);
+                if (valid) {
+#pragma unroll
+                    for (int v = 0; v < 8; ++v)
+                        part[c * 8 + v] = make_float4(
+                            __uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                            __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+                }
+            }
+            continue;
+        }
     }
     uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D);
 #pragma unroll
@@ -715,7 +738,9 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
 // ---------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------
-template <int D, int NT, int KB, bool GQ>
+// MD: the overlapping-window comparator's epilogue (window partials instead
+// of the output); the rest of the kernel is shared.
+template <int D, int NT, int KB, bool GQ, bool MD = false>
 __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using C = KCfg<D, NT, KB>;
     extern __shared__ uint8_t smem_raw[];
@@ -771,7 +796,7 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
         }
     } else {
         sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D, NT, KB, GQ>(p, bars, tmem, abort_flag, warp >> 2);
+        run_softmax<D, NT, KB, GQ, MD>(p, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();
@@ -812,6 +837,48 @@ __global__ void __launch_bounds__(256) gq_combine_kernel(const float *__restrict
     uint32_t *dst = reinterpret_cast<uint32_t *>(go + (size_t)r * D + lane * kPer);
 #pragma unroll
     for (int c = 0; c < kPer; c += 2) dst[c / 2] = sm100::pack_bf16x2(acc[c] * inv, acc[c + 1] * inv);
+}
+
+// Overlapping-window mode: the mean over the windows containing each token
+// (md_cover_range gives them along each axis). One warp per token; rh / cw hold the windows' row / column offsets in the
+// partials.
+constexpr int kMaxMdAxis = 256;
+struct MdCombineParams {
+    const float *part;
+    __nv_bfloat16 *o;
+    int H, W, Ph, Pw, mh, mw, nPh, nPw, BH, md_rows, md_tw;
+    int rh[kMaxMdAxis], cw[kMaxMdAxis];
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) md_combine_kernel(const __grid_constant__ MdCombineParams p) {
+    const long long tok = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const long long N = (long long)p.H * p.W;
+    if (tok >= (long long)p.BH * N) return;
+    const int lane = threadIdx.x & 31;
+    const int bh = (int)(tok / N), t = (int)(tok - (long long)bh * N);
+    const int r = t / p.W, c = t - (t / p.W) * p.W;
+    int pi0, pi1, pj0, pj1;
+    md_cover_range(p.nPh, p.Ph, p.mh, r, &pi0, &pi1);
+    md_cover_range(p.nPw, p.Pw, p.mw, c, &pj0, &pj1);
+    constexpr int kPer = D / 32;  // channels per lane
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+    for (int pi = pi0; pi <= pi1; ++pi) {
+        const int wr0 = imax_(0, pi * p.Ph - p.mh);
+        for (int pj = pj0; pj <= pj1; ++pj) {
+            const int wc0 = imax_(0, pj * p.Pw - p.mw);
+            const size_t prow = ((size_t)bh * p.md_rows + (p.rh[pi] + r - wr0)) * p.md_tw + (p.cw[pj] + c - wc0);
+            const float *src = p.part + prow * D + lane * kPer;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) acc[i] += src[i];
+        }
+    }
+    const float inv = 1.f / float((pi1 - pi0 + 1) * (pj1 - pj0 + 1));
+    uint32_t *dst = reinterpret_cast<uint32_t *>(p.o + (size_t)tok * D + lane * kPer);
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) dst[i / 2] = sm100::pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
 }
 
 // One block, one thread waiting on a barrier nothing arrives at: exercises the

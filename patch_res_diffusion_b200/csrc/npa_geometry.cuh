@@ -61,6 +61,14 @@ struct FwdParams {
     unsigned short patch_order[kMaxPatchOrder];  // patches by decreasing window area
     int n_cls;                       // runs of equal cost in patch_order (0: none recorded)
     int cls_rank0[kMaxCostClasses + 1];  // first patch_order index of each run; [n_cls] = n_perm
+    // Overlapping-window mode (MultiDiffusion-style comparator): the queries
+    // of a unit are its whole window, and the normalised float32 output of
+    // every window is written to md_part, window-major: window (pi, pj)
+    // starts at row md_axis_offset(pi) of a [md_rows, md_tw] token plane per
+    // batch*head and column md_axis_offset(pj) within it.
+    int md;
+    int md_rows, md_tw;              // sum of window heights / widths over the patch rows / columns
+    float *md_part;                  // [B*heads][md_rows][md_tw][d]
 };
 
 // The window's rows are walked as three segments: [seg[0], seg[1]) and
@@ -91,6 +99,25 @@ struct BlockGeom {
 __host__ __device__ inline int imin_(int a, int b) { return a < b ? a : b; }
 __host__ __device__ inline int imax_(int a, int b) { return a > b ? a : b; }
 __host__ __device__ inline int cdiv_(int a, int b) { return (a + b - 1) / b; }
+
+// Sum of the clipped window extents of the first i patches along an axis of
+// length L (patch side P, margin m).
+__host__ __device__ inline int md_axis_offset(int L, int P, int m, int i) {
+    int s = 0;
+    for (int k = 0; k < i; ++k) s += imin_(L, (k + 1) * P + m) - imax_(0, k * P - m);
+    return s;
+}
+
+__host__ __device__ inline int floor_div_(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// Overlapping-window mode: the patches (along one axis of n patches of side
+// P, margin m) whose windows contain coordinate x are [*lo, *hi]: window i
+// spans [i*P - m, (i+1)*P + m) clipped, so it contains x exactly when
+// (x - m)/P - 1 < i <= (x + m)/P.
+__host__ __device__ inline void md_cover_range(int n, int P, int m, int x, int *lo, int *hi) {
+    *lo = imax_(0, floor_div_(x - m, P));
+    *hi = imin_(n - 1, floor_div_(x + m, P));
+}
 
 // Host: key blocks a patch's clipped window needs (the scheduling cost of
 // each of its units).
@@ -154,9 +181,8 @@ inline void order_patches(FwdParams &prm) {
 // B2 h10 256x256 patch 64 margin 32 read 0.84 GB from DRAM in this order,
 // 1.13 GB with batch*head varying fastest). Without classes (more than
 // kMaxCostClasses distinct costs) batch*head varies fastest.
-__host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
-    Work w;
-    const int qb = unit % p.n_qblocks;
+// The (batch*head, patch) of a unit, in the order above.
+__host__ __device__ inline int unit_patch(const FwdParams &p, int unit, int *bh) {
     const int rest = unit / p.n_qblocks;
     int rank;
     if (p.n_cls > 0) {
@@ -164,13 +190,19 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
         while (c + 1 < p.n_cls && rest >= p.BH * p.cls_rank0[c + 1]) ++c;
         const int r = rest - p.BH * p.cls_rank0[c];
         const int cnt = p.cls_rank0[c + 1] - p.cls_rank0[c];
-        w.bh = r / cnt;
+        *bh = r / cnt;
         rank = p.cls_rank0[c] + r % cnt;
     } else {
-        w.bh = rest % p.BH;
+        *bh = rest % p.BH;
         rank = rest / p.BH;
     }
-    const int patch = p.n_perm ? int(p.patch_order[rank]) : p.patch_begin + rank;
+    return p.n_perm ? int(p.patch_order[rank]) : p.patch_begin + rank;
+}
+
+__host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
+    Work w;
+    const int qb = unit % p.n_qblocks;
+    const int patch = unit_patch(p, unit, &w.bh);
     const int pi = patch / p.nPw, pj = patch % p.nPw;
     w.pr0 = pi * p.Ph;
     w.pr1 = imin_(p.H, w.pr0 + p.Ph);
@@ -180,6 +212,12 @@ __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {
     w.wr1 = imin_(p.H, w.pr1 + p.mh);
     w.wc0 = imax_(0, w.pc0 - p.mw);
     w.wc1 = imin_(p.W, w.pc1 + p.mw);
+    if (p.md) {  // overlapping windows: every token of the window is a query
+        w.pr0 = w.wr0;
+        w.pr1 = w.wr1;
+        w.pc0 = w.wc0;
+        w.pc1 = w.wc1;
+    }
     w.tile0 = p.tiles_per_unit * qb;
     const int kc = 1 << p.kc_log2;
     w.wtc = cdiv_(w.wc1 - w.wc0, kc);

@@ -173,3 +173,35 @@ def test_global_query_validation(L):
     assert f(ws=0x70000008) == npa.NPA_ERR_MISALIGNED
     assert L.npa_global_query_workspace_size(1, 1, 8, 8, 96, 5) == 0
     assert L.npa_global_query_workspace_size(1, 1, 8, 8, 64, 0) == 0
+
+
+def test_multidiffusion_validation(L):
+    ws_ok = L.npa_multidiffusion_workspace_size(1, 1, 8, 8, 64, 4, 2)
+    f = lambda q=A, o=O_, ws=0x70000000, nb=ws_ok, patch=4, margin=2, d=64, H=8: \
+        L.npa_multidiffusion_attention_fwd(q, B_, C_, o, 1, 1, H, 8, d, patch, margin, None, ws, nb, None)
+    assert f(ws=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(ws=0x70000008) == npa.NPA_ERR_MISALIGNED
+    assert f(nb=ws_ok - 1) == npa.NPA_ERR_INVALID_ARG                 # workspace too small
+    assert f(ws=A) == npa.NPA_ERR_INVALID_ARG                         # workspace overlaps q
+    assert f(ws=O_) == npa.NPA_ERR_INVALID_ARG                        # workspace overlaps o
+    assert f(patch=0) == npa.NPA_ERR_INVALID_ARG
+    assert f(margin=-1) == npa.NPA_ERR_INVALID_ARG
+    assert f(d=96) == npa.NPA_ERR_UNSUPPORTED
+    assert f(q=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(H=300, patch=1, margin=0, nb=1 << 40) == npa.NPA_ERR_UNSUPPORTED   # 300 patch rows > 256
+    assert L.npa_multidiffusion_workspace_size(1, 1, 8, 8, 96, 4, 2) == 0
+    assert L.npa_multidiffusion_workspace_size(1, 1, 8, 8, 64, 0, 2) == 0
+
+
+@pytest.mark.parametrize("H,W,P,m,G", [(256, 256, 64, 32, 0), (40, 37, 16, 5, 7), (9, 7, 3, 2, 0),
+                                       (64, 64, 16, 0, 3)])
+def test_multidiffusion_flops_and_workspace_match_oracle_windows(H, W, P, m, G):
+    d, B, h = 64, 2, 3
+    assert npa.npa_multidiffusion_useful_flops(B, h, H, W, d, P, m, G) == \
+        4.0 * d * B * h * oracle.md_pair_count(H, W, P, m, G)
+    nph, npw = (H + P - 1) // P, (W + P - 1) // P
+    # the windows of column 0 (width min(W, P + m)) and of row 0 (height
+    # min(H, P + m)) give the per-axis extents
+    hs = [len(oracle.md_window_keys(H, W, P, m, i, 0)) // min(W, P + m) for i in range(nph)]
+    ws = [len(oracle.md_window_keys(H, W, P, m, 0, j)) // min(H, P + m) for j in range(npw)]
+    assert npa.npa_multidiffusion_workspace_size(B, h, H, W, d, P, m) == 4 * d * B * h * sum(hs) * sum(ws)

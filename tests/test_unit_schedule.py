@@ -78,3 +78,11 @@ def test_fallbacks(checker):
     assert r["ordered"] == 225 and r["classes"] == 15
     r = run(checker, *CASES["too_many_classes"], 148)
     assert r["ordered"] == 225 and r["classes"] == 0
+
+
+@pytest.mark.parametrize("L,P,m", [(256, 64, 32), (40, 16, 5), (100, 9, 3), (9, 5, 30), (37, 4, 0), (50, 7, 13)])
+def test_overlapping_window_cover_range(checker, L, P, m):
+    """The closed-form range of windows containing a coordinate (used by the
+    overlapping-window combine) equals a scan over every window."""
+    out = subprocess.run([checker, "cover", str(L), str(P), str(m)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout + out.stderr

@@ -4,7 +4,8 @@
 // (a group of tiles_per_unit query tiles) exactly once, that unit costs never increase along the order when an
 // order was built (at most kMaxPatchOrder patches), and prints the number of
 // ordered patches, the number of cost classes and the batch*head values the
-// first `wave` units touch. Built and run by test_unit_schedule.py.
+// first `wave` units touch. Built and run by test_unit_schedule.py, which
+// also runs its "cover" mode (the overlapping-window coverage rule).
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -13,7 +14,36 @@
 
 #include "../patch_res_diffusion_b200/csrc/npa_geometry.cuh"
 
+// "cover L P m": checks md_cover_range against a scan of every window along
+// an axis of length L, for every coordinate.
+static int check_cover(int L, int P, int m) {
+    const int n = (L + P - 1) / P;
+    for (int x = 0; x < L; ++x) {
+        int lo, hi, blo = -1, bhi = -1;
+        npa::md_cover_range(n, P, m, x, &lo, &hi);
+        for (int i = 0; i < n; ++i) {
+            const int w0 = i * P - m < 0 ? 0 : i * P - m, w1 = (i + 1) * P + m < L ? (i + 1) * P + m : L;
+            if (x >= w0 && x < w1) {
+                if (blo < 0) blo = i;
+                if (bhi >= 0 && bhi != i - 1) {
+                    std::printf("FAIL windows containing %d are not contiguous\n", x);
+                    return 1;
+                }
+                bhi = i;
+            }
+        }
+        if (lo != blo || hi != bhi) {
+            std::printf("FAIL x %d: range [%d, %d], scan [%d, %d]\n", x, lo, hi, blo, bhi);
+            return 1;
+        }
+    }
+    std::printf("ok cover\n");
+    return 0;
+}
+
 int main(int argc, char **argv) {
+    if (argc == 5 && std::strcmp(argv[1], "cover") == 0)
+        return check_cover(std::atoi(argv[2]), std::atoi(argv[3]), std::atoi(argv[4]));
     if (argc != 15) {
         std::fprintf(stderr, "usage: BH H W Ph Pw mh mw kb kc_log2 tiles_per_unit n_qblocks patch_begin patch_count wave\n");
         return 2;

@@ -27,7 +27,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = [
-    "Workload", "PRESETS", "preset", "f64_to_bf16_bits", "bf16_bits_to_f64",
+    "Workload", "PRESETS", "COMPARATORS", "preset", "f64_to_bf16_bits", "bf16_bits_to_f64",
     "make_inputs", "box_filter_3x3",
 ]
 
@@ -37,9 +37,11 @@ class Workload:
     """One synthetic attention workload.
 
     ``geometry`` is ``"npa"`` (square query patches of side ``patch`` with a
-    K/V window grown by ``margin`` and clipped to the grid) or ``"pcpp"``
+    K/V window grown by ``margin`` and clipped to the grid), ``"pcpp"``
     (``n_strips`` row strips, each also seeing the nearest rows of its
-    adjacent strips, the count set by the partial value ``p``).
+    adjacent strips, the count set by the partial value ``p``) or ``"md"``
+    (the overlapping-window comparator: every NPA window attends within
+    itself, outputs averaged over the windows containing a token).
     """
 
     name: str
@@ -86,8 +88,18 @@ PRESETS: Dict[str, Workload] = {
 }
 
 
+# Comparator workloads (not targets): the overlapping-window attention NPA
+# replaces, on the SDXL 4096^2 attention shape.
+COMPARATORS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("md_sdxl_4096", "md", B=2, heads=10, H=256, W=256, d=64, patch=64, margin=32),
+    ]
+}
+
+
 def preset(name: str) -> Workload:
-    return PRESETS[name]
+    return PRESETS[name] if name in PRESETS else COMPARATORS[name]
 
 
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
