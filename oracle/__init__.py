@@ -37,6 +37,7 @@ __all__ = [
     "pcpp_attention", "pcpp_attention_stale", "pair_count", "num_threads", "dense_mask",
     "dense_attention", "dense_pcpp_stale", "global_query_attention", "bf16_to_f64",
     "multidiffusion_attention", "md_window_keys", "md_window_count", "md_pair_count",
+    "asg_guidance_combine",
 ]
 
 _LIB = None
@@ -348,3 +349,26 @@ def dense_pcpp_stale(q, k, v, ks, vs, *, B, heads, H, W, d, n_strips, p, gk=None
     if G:
         out += np.einsum("bhtj,bhjc->bhtc", w[..., N:], bf16_to_f64(gv).reshape(B, heads, G, d))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Asynchronous structure guidance (ASG) combine
+# ---------------------------------------------------------------------------
+
+def asg_guidance_combine(eps, eps_ref, mask, w_t: float) -> np.ndarray:
+    """ASGDiffusion (pith.science review), "core_discovery" and
+    "key_machinery": the corrected noise of patch i is its own prediction plus
+    the guidance G_t = w_t * M * (eps_ref - eps_i), where eps_ref is the
+    reference patch's prediction from the previous step (the asynchronous
+    substitution) and M the normalised mask. Reading taken here: M is one
+    spatial map per patch and batch element, broadcast over the channels.
+
+    eps: bf16 bits [n_patches, B, C, S]; eps_ref: [B, C, S]; mask: [n_patches,
+    B, S]. Returns float64 [n_patches, B, C, S], exact up to float64 rounding.
+    """
+    e = bf16_to_f64(np.asarray(eps, dtype=np.uint16))
+    r = bf16_to_f64(np.asarray(eps_ref, dtype=np.uint16))
+    m = bf16_to_f64(np.asarray(mask, dtype=np.uint16))
+    if e.ndim != 4 or r.shape != e.shape[1:] or m.shape != (e.shape[0], e.shape[1], e.shape[3]):
+        raise ValueError("shapes: eps [n, B, C, S], eps_ref [B, C, S], mask [n, B, S]")
+    return e + float(w_t) * m[:, :, None, :] * (r[None] - e)
