@@ -31,7 +31,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import COMPARATORS, PRESETS, Workload, make_inputs, preset  # noqa: E402
+from workloads import ASG_WORKLOADS, COMPARATORS, PRESETS, AsgWorkload, Workload, make_asg_inputs, make_inputs, \
+    preset  # noqa: E402
 
 DEFAULT_WORKLOAD = "npa_sdxl_4096"
 L2_BYTES = 126 * 1024 * 1024
@@ -46,7 +47,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(PRESETS) + sorted(COMPARATORS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(PRESETS) + sorted(COMPARATORS) + sorted(ASG_WORKLOADS))
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -483,15 +485,163 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# ASG guidance combine (HBM-bound elementwise pass)
+# ---------------------------------------------------------------------------
+ASG_METRIC = "ASG guidance combine: algorithmic HBM bytes per second"
+
+
+def asg_describe(w: AsgWorkload) -> dict:
+    return {"workload": w.name, "n_patches": w.n_patches, "B": w.B, "C": w.C, "pixels_per_patch": w.S,
+            "w_t": w.w_t, "algorithmic_bytes": w.algorithmic_bytes()}
+
+
+def asg_oracle_rate(w: AsgWorkload, inp: dict, seconds: float) -> dict:
+    """Times the float64 oracle on growing leading slices of the patches."""
+    import oracle
+    n, total_b, total_t = 1, 0, 0.0
+    while total_t < seconds:
+        k = min(n, w.n_patches)
+        t0 = time.perf_counter()
+        oracle.asg_guidance_combine(inp["eps"][:k], inp["ref"], inp["mask"][:k], w.w_t)
+        total_t += time.perf_counter() - t0
+        total_b += 2 * (2 * k * w.B * w.C * w.S + k * w.B * w.S + w.B * w.C * w.S)
+        n *= 2
+    return {"value": total_b / total_t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"leading patch slices of {w.name}, float64 NumPy, {total_t:.1f} s"}
+
+
+def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+    import patch_res_diffusion_b200 as npa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    inp = make_asg_inputs(w)
+    as_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+    eps, ref, mask = as_dev(inp["eps"]), as_dev(inp["ref"]), as_dev(inp["mask"])
+    out = torch.empty_like(eps)
+    stream = torch.cuda.current_stream(dev)
+    nbytes = w.algorithmic_bytes()
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if nbytes < 2 * L2_BYTES else None
+
+    def call(e=eps, r=ref, m=mask, o=out):
+        npa.asg_guidance_combine(e, r, m, o, w.n_patches, w.B, w.C, w.S, w.w_t, stream)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.fill_(1)
+        call()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.fill_(1)
+        starts[i].record(stream)
+        call()
+        ends[i].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    timed_ms = sum(kernel_ms) if flush is not None else t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([timed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        timed_ms = float(t.item())
+    value = world * nbytes * args.steps / (timed_ms * 1e-3) / 1e9
+    avg_ms = sum(kernel_ms) / args.steps
+
+    e2e = None
+    if not args.no_e2e:
+        h_in = [x.to("cpu").pin_memory() for x in (eps, ref, mask)]
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(x.numel() * 2 for x in h_in)
+        d2h = out.numel() * 2
+
+        def e2e_step():
+            for hd, dv in zip(h_in, (eps, ref, mask)):
+                dv.copy_(hd, non_blocking=True)
+            call()
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a.elapsed_time(b)
+        e2e = {"value": world * nbytes * args.steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    achieved = nbytes / (avg_ms * 1e-3) / 1e9
+    cfg = asg_describe(w)
+    cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
+    cfg["l2"] = ("flushed (256 MB write) between launches; value from per-launch events" if flush is not None
+                 else f"inputs larger than L2 ({nbytes / 2**20:.0f} MiB per launch)")
+    line = {
+        "metric": ASG_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": timed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16 in, f32 arithmetic", "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_kind": f"{pk_kind} HBM copy",
+                     "kernel": "asg_combine_kernel", "bytes_per_launch": nbytes, "avg_launch_ms": avg_ms},
+        "cpu_baseline": None if args.no_cpu_baseline or world > 1 else asg_oracle_rate(w, inp, args.cpu_seconds),
+        "e2e": e2e, "clocks": clk, "gpu_launches": args.steps,
+        "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_asg_reference(args, w: AsgWorkload, rank: int) -> None:
+    if rank != 0:
+        return
+    inp = make_asg_inputs(w)
+    budget = max(0.5, min(2.0 * args.cpu_seconds, 30.0) / max(1, args.steps + args.warmup))
+    steps = [asg_oracle_rate(w, inp, budget) for _ in range(args.warmup + args.steps)][args.warmup:]
+    value = statistics.median(r["value"] for r in steps)
+    print(json.dumps({
+        "impl": "reference", "metric": ASG_METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.algorithmic_bytes() / (value * 1e9) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": asg_describe(w),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": steps[-1]["sample"]},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def main():
     args = parse()
-    w = preset(args.workload)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, w, rank)
-        return
+    if args.workload in ASG_WORKLOADS:
+        w = ASG_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            run_asg_reference(args, w, rank)
+            return
+        run = run_asg
+    else:
+        w = preset(args.workload)
+        if args.impl == "reference":
+            run_reference(args, w, rank)
+            return
+        run = run_ours
     if world > 1:
         import datetime
         import torch
@@ -499,7 +649,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        run_ours(args, w, rank, world, local_rank)
+        run(args, w, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

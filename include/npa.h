@@ -184,6 +184,21 @@ size_t npa_multidiffusion_workspace_size(int B, int heads, int H, int W, int d, 
  * for invalid arguments. */
 double npa_multidiffusion_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G);
 
+/* Asynchronous structure guidance combine (ASGDiffusion review,
+ * "core_discovery" and "key_machinery"): every patch's noise prediction is
+ * pulled toward the reference patch's prediction from the previous step,
+ *   out[i, b, c, s] = eps[i, b, c, s] + w_t * mask[i, b, s] * (eps_ref[b, c, s] - eps[i, b, c, s]).
+ * The pages leave the mask's layout open; here it is one spatial map per
+ * patch and batch element, shared by the channels. eps, out: bfloat16
+ * [n_patches, B, C, S] (S = latent pixels of a patch); eps_ref: [B, C, S];
+ * mask: [n_patches, B, S]; all device memory, 16-byte aligned. out may be eps
+ * itself (in place) but must not otherwise overlap an input. Arithmetic in
+ * float32 (one fused multiply-add), bf16 result rounded to nearest even.
+ * NPA_ERR_INVALID_ARG for null pointers, sizes < 1, a non-finite w_t or an
+ * overlap; NPA_ERR_MISALIGNED; NPA_ERR_UNSUPPORTED past 2^40 elements. */
+npa_status asg_guidance_combine(const void *eps, const void *eps_ref, const void *mask, void *out, int n_patches,
+                                int B, int C, int S, float w_t, npa_stream_t stream);
+
 /* Workspace bytes npa_global_query_attention_fwd uses for its full split
  * count on the current device (0: no split needed, or invalid arguments). */
 size_t npa_global_query_workspace_size(int B, int heads, int H, int W, int d, int G);

@@ -31,7 +31,7 @@ __all__ = [
     "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "npa_global_query_attention_fwd",
     "npa_global_query_workspace_size", "npa_global_query_attention_fwd_noalloc", "global_query_attention",
     "npa_multidiffusion_attention_fwd", "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops",
-    "multidiffusion_attention", "EXPORTED_SYMBOLS",
+    "multidiffusion_attention", "asg_guidance_combine", "asg_combine", "EXPORTED_SYMBOLS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
@@ -48,7 +48,7 @@ EXPORTED_SYMBOLS = (
     "pcpp_useful_flops", "npa_device_status", "npa_selftest_wait_timeout", "npa_status_string",
     "npa_global_query_attention_fwd", "npa_global_query_workspace_size",
     "npa_global_query_attention_fwd_noalloc", "npa_multidiffusion_attention_fwd",
-    "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops",
+    "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops", "asg_guidance_combine",
 )
 
 
@@ -91,6 +91,8 @@ def lib() -> ctypes.CDLL:
         L.npa_multidiffusion_workspace_size.restype = ctypes.c_size_t
         L.npa_multidiffusion_useful_flops.argtypes = [i] * 8
         L.npa_multidiffusion_useful_flops.restype = d
+        L.asg_guidance_combine.argtypes = [vp] * 4 + [i] * 4 + [ctypes.c_float, vp]
+        L.asg_guidance_combine.restype = i
         L.npa_global_query_workspace_size.argtypes = [i] * 6
         L.npa_global_query_workspace_size.restype = ctypes.c_size_t
         L.pcpp_neighbor_rows.argtypes = [i, d]
@@ -206,6 +208,14 @@ def npa_multidiffusion_useful_flops(B, heads, H, W, d, patch, margin, G=0) -> fl
     return float(lib().npa_multidiffusion_useful_flops(B, heads, H, W, d, patch, margin, G))
 
 
+def asg_guidance_combine(eps, eps_ref, mask, out, n_patches: int, B: int, C: int, S: int, w_t: float,
+                         stream=None) -> None:
+    """C ``asg_guidance_combine``: out = eps + w_t * mask * (eps_ref - eps)."""
+    _check(lib().asg_guidance_combine(_ptr(eps), _ptr(eps_ref), _ptr(mask), _ptr(out), n_patches, B, C, S,
+                                      float(w_t), _stream(stream)),
+           "asg_guidance_combine")
+
+
 def npa_global_query_workspace_size(B, heads, H, W, d, G) -> int:
     return int(lib().npa_global_query_workspace_size(B, heads, H, W, d, G))
 
@@ -314,4 +324,14 @@ def multidiffusion_attention(q, k, v, H: int, W: int, patch: int, margin: int, g
     G = 0 if global_k is None else int(global_k.shape[2])
     npa_multidiffusion_attention_fwd(q, k, v, out, B, heads, H, W, d, patch, margin, workspace,
                                      workspace.numel() * workspace.element_size(), global_k, global_v, G, stream)
+    return out
+
+
+def asg_combine(eps, eps_ref, mask, w_t: float, out=None, stream=None):
+    """ASG combine on torch bf16 CUDA tensors: eps [n, B, C, S], eps_ref
+    [B, C, S], mask [n, B, S]; ``out=eps`` works in place."""
+    n, B, C, S = (int(x) for x in eps.shape)
+    if out is None:
+        out = eps.new_empty(eps.shape)
+    asg_guidance_combine(eps, eps_ref, mask, out, n, B, C, S, w_t, stream)
     return out

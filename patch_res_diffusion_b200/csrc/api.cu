@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "npa.h"
+#include "asg_combine.cuh"
 #include "npa_fwd_kernel.cuh"
 
 namespace {
@@ -679,6 +680,41 @@ double npa_multidiffusion_useful_flops(int B, int heads, int H, int W, int d, in
         s2c += w * w;
     }
     return 4.0 * d * (double)B * heads * (s2r * s2c + G * s1r * s1c);
+}
+
+npa_status asg_guidance_combine(const void *eps, const void *eps_ref, const void *mask, void *out, int n_patches,
+                                int B, int C, int S, float w_t, npa_stream_t stream) {
+    if (!eps || !eps_ref || !mask || !out) return NPA_ERR_INVALID_ARG;
+    if (n_patches < 1 || B < 1 || C < 1 || S < 1 || !std::isfinite(w_t)) return NPA_ERR_INVALID_ARG;
+    if (!aligned16(eps) || !aligned16(eps_ref) || !aligned16(mask) || !aligned16(out)) return NPA_ERR_MISALIGNED;
+    const long long nb = (long long)n_patches * B;
+    if (nb * C > (1LL << 40) / S || nb > INT_MAX) return NPA_ERR_UNSUPPORTED;
+    const size_t e_bytes = (size_t)nb * C * S * 2, r_bytes = (size_t)B * C * S * 2, m_bytes = (size_t)nb * S * 2;
+    if (out != eps && overlaps(out, e_bytes, eps, e_bytes)) return NPA_ERR_INVALID_ARG;
+    if (overlaps(out, e_bytes, eps_ref, r_bytes) || overlaps(out, e_bytes, mask, m_bytes)) return NPA_ERR_INVALID_ARG;
+    int sm_count = 0;
+    const npa_status st = ensure_ready(&sm_count);
+    if (st != NPA_OK) return st;
+    npa::AsgParams prm;
+    prm.eps = static_cast<const __nv_bfloat16 *>(eps);
+    prm.ref = static_cast<const __nv_bfloat16 *>(eps_ref);
+    prm.mask = static_cast<const __nv_bfloat16 *>(mask);
+    prm.out = static_cast<__nv_bfloat16 *>(out);
+    prm.B = B;
+    prm.C = C;
+    prm.S = S;
+    prm.chunks = (S + 7) / 8;
+    prm.n_items = nb * prm.chunks;
+    prm.w = w_t;
+    prm.vec = S % 8 == 0;
+    // enough blocks for every chunk, at most 8 resident 256-thread blocks per
+    // multiprocessor (the kernel strides over the rest)
+    const long long blocks = (prm.n_items + 255) / 256;
+    const unsigned grid = (unsigned)(blocks < 8LL * sm_count ? blocks : 8LL * sm_count);
+    void *args[1] = {&prm};
+    const cudaError_t e =
+        cudaLaunchKernel((const void *)npa::asg_combine_kernel, dim3(grid), dim3(256), args, 0, (cudaStream_t)stream);
+    return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
 }
 
 int pcpp_neighbor_rows(int strip_rows, double p) { return neighbor_rows(strip_rows, p); }

@@ -205,3 +205,18 @@ def test_multidiffusion_flops_and_workspace_match_oracle_windows(H, W, P, m, G):
     hs = [len(oracle.md_window_keys(H, W, P, m, i, 0)) // min(W, P + m) for i in range(nph)]
     ws = [len(oracle.md_window_keys(H, W, P, m, 0, j)) // min(H, P + m) for j in range(npw)]
     assert npa.npa_multidiffusion_workspace_size(B, h, H, W, d, P, m) == 4 * d * B * h * sum(hs) * sum(ws)
+
+
+def test_asg_validation(L):
+    f = lambda eps=A, ref=B_, m=C_, out=O_, n=2, B=1, C=4, S=64, w=1.5: \
+        L.asg_guidance_combine(eps, ref, m, out, n, B, C, S, w, None)
+    assert f(eps=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(out=None) == npa.NPA_ERR_INVALID_ARG
+    assert f(n=0) == npa.NPA_ERR_INVALID_ARG
+    assert f(S=0) == npa.NPA_ERR_INVALID_ARG
+    assert f(w=float("nan")) == npa.NPA_ERR_INVALID_ARG
+    assert f(w=float("inf")) == npa.NPA_ERR_INVALID_ARG
+    assert f(m=C_ + 2) == npa.NPA_ERR_MISALIGNED
+    assert f(out=A + 16) == npa.NPA_ERR_INVALID_ARG        # partly overlaps eps (only exact in-place is allowed)
+    assert f(out=B_) == npa.NPA_ERR_INVALID_ARG            # overlaps the reference
+    assert f(out=C_) == npa.NPA_ERR_INVALID_ARG            # overlaps the mask

@@ -27,7 +27,7 @@ from typing import Dict, Optional
 import numpy as np
 
 __all__ = [
-    "Workload", "PRESETS", "COMPARATORS", "preset", "f64_to_bf16_bits", "bf16_bits_to_f64",
+    "Workload", "PRESETS", "COMPARATORS", "preset", "AsgWorkload", "ASG_WORKLOADS", "make_asg_inputs", "f64_to_bf16_bits", "bf16_bits_to_f64",
     "make_inputs", "box_filter_3x3",
 ]
 
@@ -171,3 +171,47 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray
         out["gk"] = f64_to_bf16_bits(_normal(s + 3, gshape))
         out["gv"] = f64_to_bf16_bits(_normal(s + 4, gshape))
     return out
+
+
+@dataclasses.dataclass(frozen=True)
+class AsgWorkload:
+    """One synthetic ASG guidance-combine workload: ``n_patches`` latent
+    patches of ``S`` pixels and ``C`` channels for ``B`` batch elements, one
+    reference patch, one mask per patch, weight ``w_t``."""
+
+    name: str
+    n_patches: int
+    B: int
+    C: int
+    S: int
+    w_t: float = 0.8
+    seed: int = 0
+
+    @property
+    def elements(self) -> int:
+        return self.n_patches * self.B * self.C * self.S
+
+    def algorithmic_bytes(self) -> int:
+        """eps read and out written once, the mask read once, the reference once."""
+        return 2 * (2 * self.elements + self.n_patches * self.B * self.S + self.B * self.C * self.S)
+
+
+# SDXL at 4096^2: a 512^2 x 4 latent cut into 16 patches of the model's
+# native 128^2 latent size, classifier-free guidance batch 2. The bulk case
+# streams ~1.2 GB through the same kernel to measure its bandwidth.
+ASG_WORKLOADS: Dict[str, AsgWorkload] = {
+    w.name: w
+    for w in [
+        AsgWorkload("asg_sdxl_4096", n_patches=16, B=2, C=4, S=128 * 128),
+        AsgWorkload("asg_bulk", n_patches=16, B=8, C=16, S=256 * 256),
+    ]
+}
+
+
+def make_asg_inputs(w: AsgWorkload) -> Dict[str, np.ndarray]:
+    """eps and the reference ~ N(0, 1), the mask ~ U[0, 1), as bf16 bits (seeds
+    seed + 0, 1, 2)."""
+    eps = f64_to_bf16_bits(_normal(w.seed, (w.n_patches, w.B, w.C, w.S)))
+    ref = f64_to_bf16_bits(_normal(w.seed + 1, (w.B, w.C, w.S)))
+    mask = f64_to_bf16_bits(np.random.default_rng(w.seed + 2).uniform(0.0, 1.0, (w.n_patches, w.B, w.S)))
+    return {"eps": eps, "ref": ref, "mask": mask}
