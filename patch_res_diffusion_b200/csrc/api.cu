@@ -13,6 +13,7 @@
 
 #include "npa.h"
 #include "asg_combine.cuh"
+#include "md_combine.cuh"
 #include "npa_fwd_kernel.cuh"
 
 namespace {
@@ -367,7 +368,8 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
         for (int j = 0; j < prm.nPw; ++j) cp.cw[j] = npa::md_axis_offset(g.W, g.Pw, g.mw, j);
         void *cargs[1] = {&cp};
         const long long tokens = (long long)BH * g.H * g.W;
-        const dim3 cgrid((unsigned)((tokens + 7) / 8));
+        const long long per_block = 256 / (d / 4);  // tokens per 256-thread block
+        const dim3 cgrid((unsigned)((tokens + per_block - 1) / per_block));
         if (d == 64)
             e = cudaLaunchKernel((const void *)npa::md_combine_kernel<64>, cgrid, dim3(256), cargs, 0,
                                  (cudaStream_t)stream);

@@ -839,48 +839,6 @@ __global__ void __launch_bounds__(256) gq_combine_kernel(const float *__restrict
     for (int c = 0; c < kPer; c += 2) dst[c / 2] = sm100::pack_bf16x2(acc[c] * inv, acc[c + 1] * inv);
 }
 
-// Overlapping-window mode: the mean over the windows containing each token
-// (md_cover_range gives them along each axis). One warp per token; rh / cw hold the windows' row / column offsets in the
-// partials.
-constexpr int kMaxMdAxis = 256;
-struct MdCombineParams {
-    const float *part;
-    __nv_bfloat16 *o;
-    int H, W, Ph, Pw, mh, mw, nPh, nPw, BH, md_rows, md_tw;
-    int rh[kMaxMdAxis], cw[kMaxMdAxis];
-};
-
-template <int D>
-__global__ void __launch_bounds__(256) md_combine_kernel(const __grid_constant__ MdCombineParams p) {
-    const long long tok = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const long long N = (long long)p.H * p.W;
-    if (tok >= (long long)p.BH * N) return;
-    const int lane = threadIdx.x & 31;
-    const int bh = (int)(tok / N), t = (int)(tok - (long long)bh * N);
-    const int r = t / p.W, c = t - (t / p.W) * p.W;
-    int pi0, pi1, pj0, pj1;
-    md_cover_range(p.nPh, p.Ph, p.mh, r, &pi0, &pi1);
-    md_cover_range(p.nPw, p.Pw, p.mw, c, &pj0, &pj1);
-    constexpr int kPer = D / 32;  // channels per lane
-    float acc[kPer];
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
-    for (int pi = pi0; pi <= pi1; ++pi) {
-        const int wr0 = imax_(0, pi * p.Ph - p.mh);
-        for (int pj = pj0; pj <= pj1; ++pj) {
-            const int wc0 = imax_(0, pj * p.Pw - p.mw);
-            const size_t prow = ((size_t)bh * p.md_rows + (p.rh[pi] + r - wr0)) * p.md_tw + (p.cw[pj] + c - wc0);
-            const float *src = p.part + prow * D + lane * kPer;
-#pragma unroll
-            for (int i = 0; i < kPer; ++i) acc[i] += src[i];
-        }
-    }
-    const float inv = 1.f / float((pi1 - pi0 + 1) * (pj1 - pj0 + 1));
-    uint32_t *dst = reinterpret_cast<uint32_t *>(p.o + (size_t)tok * D + lane * kPer);
-#pragma unroll
-    for (int i = 0; i < kPer; i += 2) dst[i / 2] = sm100::pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-}
-
 // One block, one thread waiting on a barrier nothing arrives at: exercises the
 // bounded-wait path and the status word without touching the GPU's health.
 __global__ void npa_wait_selftest_kernel(unsigned long long limit_ns) {
