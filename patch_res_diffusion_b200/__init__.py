@@ -12,10 +12,22 @@ a call fails, an exception is raised.
 * ``pcpp_attention_fwd`` - partially conditioned attention (PCPP review, "What
   carries the argument"): row strips attending to themselves plus the nearest
   ceil(p * rows) rows of each adjacent strip.
+* ``pcpp_attention_fwd_stale`` - PCPP as it runs across devices (PCPP review,
+  "Core claim"): the strip's own keys from the current step, the borrowed
+  neighbour rows from the previous step's keys/values.
+* ``npa_global_query_attention_fwd`` (and ``..._noalloc``) - the text-query
+  half of joint attention: global tokens as queries over all keys.
 * ``npa_multidiffusion_attention_fwd`` - the overlapping-window comparator
   (ScaleDiff summary, "Approach": MultiDiffusion averages overlapping
   patches): each NPA window attends within itself and a token's output is the
   mean over the windows that contain it.
+* ``asg_guidance_combine`` - asynchronous structure guidance (ASGDiffusion
+  review, "core_discovery"): eps + w_t * M * (eps_ref - eps) per patch.
+
+The lower-case helpers (``npa_attention``, ``pcpp_attention``,
+``pcpp_attention_stale``, ``global_query_attention``,
+``multidiffusion_attention``, ``asg_combine``) take torch CUDA tensors and
+allocate outputs and workspaces; the computation is the same C call.
 """
 from __future__ import annotations
 
