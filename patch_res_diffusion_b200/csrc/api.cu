@@ -1,6 +1,6 @@
 // api.cu - host side of the C ABI declared in include/npa.h: argument
-// validation, geometry resolution, TMA tensor-map encoding and the launch of
-// the sm_100a kernel. Nothing here computes attention.
+// validation, geometry resolution, TMA tensor-map encoding and the launches of
+// the sm_100a kernels. Nothing here computes attention or the combines.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -3,9 +3,8 @@
 //
 // A persistent CTA works through units of NT query tiles (128 queries each) of
 // one patch that share the patch's key/value window, streamed in blocks of KB
-// keys. Two shapes are instantiated:
-//   NT = 3, KB = 64  (image-token queries at d = 64)
-//   NT = 2, KB = 128 (d = 128, and the global-token queries)
+// keys. Every path runs NT = 2, KB = 128; NT = 3, KB = 64 (three softmax
+// warpgroups at d = 64) is a build option of the host launcher.
 // Warps (NT + 1 warpgroups):
 //   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes 0..127)
 //   control warp 0     TMA producer (Q once per unit, then K and V blocks
