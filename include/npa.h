@@ -44,6 +44,15 @@
  * a lock on first use, so the entry points are safe to call from several host
  * threads.
  *
+ * CUDA graphs: after a first call on a device (which checks the device and
+ * sets kernel attributes), npa_attention_fwd, pcpp_attention_fwd,
+ * pcpp_attention_fwd_stale, npa_global_query_attention_fwd,
+ * npa_multidiffusion_attention_fwd and asg_guidance_combine may be captured in
+ * a stream capture. The tensor maps are encoded on the host when the call is
+ * captured, so the graph replays on the same buffers (their contents may
+ * change between replays); npa_device_status synchronises and must not be
+ * captured.
+ *
  * Errors: every entry point validates its arguments on the host and returns a
  * status code; nothing aborts, prints or throws across this boundary. A
  * failed launch returns NPA_ERR_CUDA. Device-side waits are bounded; if one

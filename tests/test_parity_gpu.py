@@ -183,3 +183,48 @@ def test_bounded_wait_reports_timeout():
     npa.npa_selftest_wait_timeout(2000)
     assert npa.npa_device_status() == npa.NPA_ERR_DEVICE_TIMEOUT
     assert npa.npa_device_status() == npa.NPA_OK  # read clears it
+
+
+@pytest.mark.parametrize("kind", ["npa_d64", "pcpp_d128_global", "global_query_split", "multidiffusion"])
+def test_cuda_graph_replay(kind):
+    """Once a first call has set the device up, a call can be captured in a
+    CUDA graph: the tensor maps are encoded on the host at capture time and
+    the graph replays the launches on the same buffers. Replays must equal
+    eager calls bit for bit, also after the inputs are overwritten in place."""
+    import patch_res_diffusion_b200 as npa
+    rng = np.random.default_rng(11)
+    r = lambda *shape: to_device(f64_to_bf16_bits(rng.standard_normal(shape)))
+    if kind == "npa_d64":
+        H, W, args = 24, 40, dict(patch=8, margin=4)
+        q, k, v = r(1, 2, H * W, 64), r(1, 2, H * W, 64), r(1, 2, H * W, 64)
+        call = lambda out: npa.npa_attention(q, k, v, H, W, out=out, **args)
+    elif kind == "pcpp_d128_global":
+        H, W = 32, 24
+        q, k, v, gk, gv = r(1, 2, H * W, 128), r(1, 2, H * W, 128), r(1, 2, H * W, 128), r(1, 2, 9, 128), \
+            r(1, 2, 9, 128)
+        call = lambda out: npa.pcpp_attention(q, k, v, H, W, 4, 0.3, gk, gv, out=out)
+    elif kind == "global_query_split":
+        H, W = 16, 16
+        q, k, v, gk, gv = r(1, 4, 130, 64), r(1, 4, H * W, 64), r(1, 4, H * W, 64), r(1, 4, 130, 64), \
+            r(1, 4, 130, 64)
+        call = lambda out: npa.global_query_attention(q, k, v, gk, gv, H, W, out=out, split=True)
+    else:
+        H, W = 20, 24
+        q, k, v = r(1, 2, H * W, 64), r(1, 2, H * W, 64), r(1, 2, H * W, 64)
+        call = lambda out: npa.multidiffusion_attention(q, k, v, H, W, 8, 3, out=out)
+    eager = call(torch.empty_like(q))
+    out = torch.full_like(q, float("nan"))
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        call(out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    q.copy_(r(*q.shape))                        # new queries, same buffer
+    eager2 = call(torch.empty_like(q))
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager2.view(torch.int16))
+    assert not torch.equal(eager.view(torch.int16), eager2.view(torch.int16))
