@@ -74,6 +74,12 @@ def test_null_and_size_arguments_rejected(L):
     assert _pcpp(L, n=0) == npa.NPA_ERR_INVALID_ARG
 
 
+def test_sizes_past_the_tensor_map_limits_rejected(L):
+    # a 2^20 x 2^20 grid at d = 64 needs 2^47-byte row strides: refused before any CUDA call
+    assert _npa(L, H=1 << 20, W=1 << 20) == npa.NPA_ERR_UNSUPPORTED
+    assert _pcpp(L, H=1 << 20, W=1 << 20, n=1) == npa.NPA_ERR_UNSUPPORTED
+
+
 def test_unsupported_head_dim(L):
     for d in (16, 32, 96, 256):
         assert _npa(L, d=d) == npa.NPA_ERR_UNSUPPORTED

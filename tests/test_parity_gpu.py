@@ -63,6 +63,28 @@ def test_small_full_parity(w):
     assert passes(m), m
 
 
+# Degenerate geometries: every token its own patch, a single token, one
+# column, one row, a grid much smaller than the global-token set, one-row
+# strips.
+EDGE = [
+    Workload("npa_patch1", "npa", B=1, heads=2, H=12, W=10, d=64, patch=1, margin=1),
+    Workload("npa_single_token", "npa", B=2, heads=1, H=1, W=1, d=64, patch=1, margin=0),
+    Workload("npa_one_column", "npa", B=1, heads=2, H=50, W=1, d=64, patch=8, margin=3),
+    Workload("npa_one_row_d128", "npa", B=1, heads=1, H=1, W=77, d=128, patch=16, margin=5),
+    Workload("npa_tiny_grid_many_global", "npa", B=1, heads=2, H=2, W=3, d=64, patch=2, margin=1, G=300),
+    Workload("pcpp_one_row_strips", "pcpp", B=1, heads=2, H=16, W=40, d=64, n_strips=16, p=1.0),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=lambda w: w.name)
+def test_degenerate_geometries(w):
+    inp = make_inputs(w)
+    got = to_f64(run_gpu(w, inp))
+    m = compare(got, run_oracle(w, inp))
+    log_metrics(w.name, m)
+    assert passes(m), m
+
+
 @pytest.mark.parametrize("name", list(PRESETS))
 def test_full_workload_sampled_parity(name):
     w = PRESETS[name]
