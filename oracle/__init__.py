@@ -25,7 +25,6 @@ pages are silent):
 from __future__ import annotations
 
 import ctypes
-import os
 from typing import Optional, Sequence
 
 import numpy as np

@@ -23,7 +23,7 @@ attention arithmetic.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Tuple
+from typing import List, Tuple
 
 __all__ = ["strip_range", "neighbor_rows", "exchange_borrowed_rows", "exchange_bytes", "allgather_bytes"]
 

@@ -2,7 +2,6 @@
 declares, validates arguments before touching a GPU, and its geometry helpers
 agree with the oracle's brute-force counts. No compute call is made here."""
 import ctypes
-import math
 import os
 import re
 import subprocess

@@ -3,7 +3,6 @@ range of strips, exchanges its boundary rows with its neighbours, and runs the
 two-source oracle for its strips. Exchanging the current step's rows and
 using them at once is the synchronous limit, so the ranks' outputs must equal
 the single-process single-source PCPP oracle exactly."""
-import os
 import socket
 
 import numpy as np

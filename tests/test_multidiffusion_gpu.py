@@ -2,11 +2,10 @@
 against the float64 oracle: every NPA window attends within itself and a
 token's output is the mean over the windows containing it. Small grids are
 compared in full; the SDXL attention shapes on sampled queries."""
-import numpy as np
 import pytest
 
 import oracle
-from workloads import Workload, f64_to_bf16_bits, make_inputs
+from workloads import Workload, make_inputs
 from _parity import compare, log_metrics, passes, sample_queries, to_device, to_f64
 
 pytestmark = pytest.mark.gpu

@@ -8,8 +8,6 @@ a fixed array inside the library. These tests call it through the C ABI and
 check it against the entry point that takes a caller workspace, on two
 calls in a row (the array keeps the previous call's contents), and that
 problems too large for the array are refused. This file is collected last."""
-import ctypes
-
 import numpy as np
 import pytest
 
