@@ -62,6 +62,8 @@ def describe(w: Workload) -> dict:
         cfg.update({"geometry": w.geometry, "patch": w.patch, "margin": w.margin})
         if w.geometry == "md":
             cfg["comparator"] = "overlapping NPA windows, each attending within itself, outputs averaged"
+    elif w.geometry == "gq":
+        cfg.update({"geometry": "gq", "queries": "the global tokens, over all image and global keys"})
     else:
         cfg.update({"geometry": "pcpp", "n_strips": w.n_strips, "p": w.p})
     cfg["global_tokens"] = w.G
@@ -108,6 +110,8 @@ def useful_flops(w: Workload) -> float:
         return npa.npa_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
     if w.geometry == "md":
         return npa.npa_multidiffusion_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin, w.G)
+    if w.geometry == "gq":
+        return 4.0 * w.d * w.B * w.heads * w.G * (w.H * w.W + w.G)
     return npa.pcpp_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, w.G)
 
 
@@ -125,7 +129,17 @@ def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
         dict(n_strips=w.n_strips, p=w.p)
     fn = {"npa": oracle.npa_attention, "md": oracle.multidiffusion_attention}.get(w.geometry,
                                                                                   oracle.pcpp_attention)
-    if w.geometry == "npa":
+    if w.geometry == "pcpp_stale":
+        fn = lambda q, k, v, **kw: oracle.pcpp_attention_stale(q, k, v, inp["ks"], inp["vs"], **kw)
+    if w.geometry == "gq":
+        N_img = N
+        N = w.G  # the queries are the global tokens
+        fn = lambda q, k, v, gk, gv, G, queries, **kw: oracle.global_query_attention(
+            inp["gq"], k, v, gk, gv, G=G, queries=queries, **{a: kw[a] for a in ("B", "heads", "H", "W", "d")})
+        geom = {}
+    if w.geometry == "gq":
+        key_count = lambda t: N_img
+    elif w.geometry == "npa":
         key_count = lambda t: len(oracle.npa_key_set(w.H, w.W, w.patch, w.margin, t))
     elif w.geometry == "md":
         key_count = lambda t: md_query_pairs(w, t) - w.G * md_cover(w, t)
@@ -215,10 +229,12 @@ def run_reference(args, w: Workload, rank: int) -> None:
 
 def useful_flops_host(w: Workload) -> float:
     import oracle
+    if w.geometry == "gq":
+        return 4.0 * w.d * w.B * w.heads * w.G * (w.H * w.W + w.G)
     if w.geometry == "md":
         return 4.0 * w.d * w.B * w.heads * oracle.md_pair_count(w.H, w.W, w.patch, w.margin, w.G)
-    pairs = oracle.pair_count(w.geometry, w.H, w.W, patch=w.patch, margin=w.margin, n_strips=w.n_strips,
-                              p=w.p, G=w.G)
+    pairs = oracle.pair_count("pcpp" if w.geometry == "pcpp_stale" else w.geometry, w.H, w.W, patch=w.patch,
+                              margin=w.margin, n_strips=w.n_strips, p=w.p, G=w.G)
     return 4.0 * w.d * w.B * w.heads * pairs
 
 
@@ -300,16 +316,27 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     q, k, v = dev_bf16(inp["q"]), dev_bf16(inp["k"]), dev_bf16(inp["v"])
     gk = dev_bf16(inp["gk"]) if w.G else None
     gv = dev_bf16(inp["gv"]) if w.G else None
-    o = torch.empty_like(q)
+    ks = dev_bf16(inp["ks"]) if w.geometry == "pcpp_stale" else None
+    vs = dev_bf16(inp["vs"]) if w.geometry == "pcpp_stale" else None
+    gq = dev_bf16(inp["gq"]) if w.geometry == "gq" else None
+    o = torch.empty_like(gq if gq is not None else q)
     stream = torch.cuda.current_stream(dev)
     flops = useful_flops(w)
+    # minimum HBM bytes of one call: every input read once, the output written once
     bytes_io = (q.numel() * 4 + (2 * gk.numel() if w.G else 0)) * 2  # q, k, v, o (+ global k, v)
+    if w.geometry == "gq":  # global queries and output, global k, v, image k, v
+        bytes_io = (4 * gq.numel() + 2 * k.numel()) * 2
+    elif w.geometry == "pcpp_stale":  # + the borrowed rows of the previous step's k, v
+        r = npa.pcpp_neighbor_rows(w.H // w.n_strips, w.p)
+        bytes_io += 2 * (2 * r * (w.n_strips - 1)) * w.W * w.d * 2 * w.B * w.heads
     needs_flush = bytes_io < 2 * L2_BYTES
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if needs_flush else None
 
     md_bytes = npa.npa_multidiffusion_workspace_size(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin) \
         if w.geometry == "md" else 0
     md_ws = [torch.empty(md_bytes, dtype=torch.uint8, device=dev) for _ in range(2)] if md_bytes else None
+    gq_bytes = npa.npa_global_query_workspace_size(w.B, w.heads, w.H, w.W, w.d, w.G) if gq is not None else 0
+    gq_ws = torch.empty(max(gq_bytes, 16), dtype=torch.uint8, device=dev) if gq is not None else None
 
     def call():
         if w.geometry == "npa":
@@ -317,6 +344,12 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         elif w.geometry == "md":
             npa.npa_multidiffusion_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin,
                                                  md_ws[0], md_bytes, gk, gv, w.G, stream)
+        elif w.geometry == "pcpp_stale":
+            npa.pcpp_attention_fwd_stale(q, k, v, ks, vs, o, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, 0,
+                                         w.n_strips, gk, gv, w.G, stream)
+        elif w.geometry == "gq":
+            npa.npa_global_query_attention_fwd(gq, k, v, gk, gv, o, w.B, w.heads, w.H, w.W, w.d, w.G, gq_ws,
+                                               gq_bytes, stream)
         else:
             npa.pcpp_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, gk, gv, w.G, stream)
 
@@ -370,7 +403,7 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     # over three streams with double-buffered device tensors, so step i+1's
     # upload overlaps step i's kernel and step i-1's download.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and w.geometry in ("npa", "pcpp", "md"):
         hq, hk, hv = (x.to("cpu").pin_memory() for x in (q, k, v))
         hg = [x.to("cpu").pin_memory() for x in (gk, gv)] if w.G else []
         hos = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for _ in range(2)]
@@ -448,8 +481,9 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "peak_kind": f"{pk_kind} bf16 burst",
         "frac_of_sustained": achieved / pk["bf16_tflops_sustained"],
         "frac_of_datasheet_dense": achieved / DATASHEET_BF16_DENSE_TFLOPS,
-        "kernel": KERNEL_NAME if w.geometry != "md" else
-        KERNEL_NAME + " + md_combine_kernel (timed together: one call)", "useful_flops_per_launch": flops,
+        "kernel": {"md": KERNEL_NAME + " + md_combine_kernel (timed together: one call)",
+                   "gq": KERNEL_NAME + " + gq_combine_kernel (timed together: one call)"}.get(w.geometry, KERNEL_NAME),
+        "useful_flops_per_launch": flops,
         "avg_launch_ms": avg_kernel_ms,
         "hbm_min_bytes_per_launch": bytes_io,
     }
@@ -479,7 +513,7 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk,
-        "gpu_launches": args.steps * (2 if w.geometry == "md" else 1),
+        "gpu_launches": args.steps * (2 if w.geometry == "md" or gq_bytes > 0 else 1),
         "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
     }
     print(json.dumps(line), flush=True)

@@ -39,9 +39,11 @@ class Workload:
     ``geometry`` is ``"npa"`` (square query patches of side ``patch`` with a
     K/V window grown by ``margin`` and clipped to the grid), ``"pcpp"``
     (``n_strips`` row strips, each also seeing the nearest rows of its
-    adjacent strips, the count set by the partial value ``p``) or ``"md"``
-    (the overlapping-window comparator: every NPA window attends within
-    itself, outputs averaged over the windows containing a token).
+    adjacent strips, the count set by the partial value ``p``), ``"md"`` (the
+    overlapping-window comparator: every NPA window attends within itself,
+    outputs averaged over the windows containing a token), ``"pcpp_stale"``
+    (PCPP with the borrowed rows read from a second, previous-step K/V) or
+    ``"gq"`` (the G global tokens as queries over all image and global keys).
     """
 
     name: str
@@ -88,12 +90,16 @@ PRESETS: Dict[str, Workload] = {
 }
 
 
-# Comparator workloads (not targets): the overlapping-window attention NPA
-# replaces, on the SDXL 4096^2 attention shape.
+# Workloads of the later rows (not the throughput targets): the
+# overlapping-window comparator on the SDXL 4096^2 attention shape, PCPP with
+# stale neighbour rows on the PCPP 4x32 shape, and the text-query half of FLUX
+# 4096^2 joint attention.
 COMPARATORS: Dict[str, Workload] = {
     w.name: w
     for w in [
         Workload("md_sdxl_4096", "md", B=2, heads=10, H=256, W=256, d=64, patch=64, margin=32),
+        Workload("pcpp_stale_4x32_p0.3", "pcpp_stale", B=2, heads=10, H=128, W=128, d=64, n_strips=4, p=0.3),
+        Workload("gq_flux_4096", "gq", B=1, heads=24, H=256, W=256, d=128, G=512),
     ]
 }
 
@@ -155,7 +161,8 @@ def _normal(seed: int, shape) -> np.ndarray:
 
 
 def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
-    """Draw the q, k, v (and global gk, gv) tensors of a workload as bf16 bits."""
+    """Draw the q, k, v (and global gk, gv) tensors of a workload as bf16
+    bits; stale-row PCPP adds ks, vs and the global-query form adds gq."""
     s = w.seed if seed is None else seed
     shape = (w.B, w.heads, w.n_tokens, w.d)
     out: Dict[str, np.ndarray] = {}
@@ -170,6 +177,11 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray
         gshape = (w.B, w.heads, w.G, w.d)
         out["gk"] = f64_to_bf16_bits(_normal(s + 3, gshape))
         out["gv"] = f64_to_bf16_bits(_normal(s + 4, gshape))
+    if w.geometry == "pcpp_stale":  # the previous step's keys / values
+        out["ks"] = f64_to_bf16_bits(_normal(s + 5, shape))
+        out["vs"] = f64_to_bf16_bits(_normal(s + 6, shape))
+    if w.geometry == "gq":  # the global tokens' own queries
+        out["gq"] = f64_to_bf16_bits(_normal(s + 7, (w.B, w.heads, w.G, w.d)))
     return out
 
 
