@@ -115,6 +115,26 @@ def useful_flops(w: Workload) -> float:
     return npa.pcpp_useful_flops(w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, w.G)
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's timed region (every rank takes part; world 1 returns
+    ms). ``device``: where the reduction tensor lives (cuda under NCCL, cpu
+    under gloo)."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, slowest_ms: float) -> float:
+    """Units per second of the whole job: every rank processed
+    ``units_per_rank_step`` per step (replicas: weak scaling), over the
+    slowest rank's time."""
+    return world * units_per_rank_step * steps / (slowest_ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload)
 # ---------------------------------------------------------------------------
@@ -391,11 +411,8 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     kernel_ms_sum = sum(kernel_ms)
     elapsed_ms = t_begin.elapsed_time(t_end)
     timed_ms = kernel_ms_sum if flush is not None else elapsed_ms
-    if world > 1:
-        t = torch.tensor([timed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        timed_ms = float(t.item())
-    value = world * flops * args.steps / (timed_ms * 1e-3) / 1e12
+    timed_ms = max_over_ranks(timed_ms, world, dev)
+    value = whole_job_rate(world, flops, args.steps, timed_ms) / 1e12
     avg_kernel_ms = kernel_ms_sum / args.steps
 
     # End to end through host buffers: every step copies its inputs from pinned
@@ -460,11 +477,8 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         e1.record(s_out)
         torch.cuda.synchronize(dev)
         e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * flops * args.steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e_ms, world, dev)
+        e2e = {"value": whole_job_rate(world, flops, args.steps, e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps,
                "pipelined": "upload / kernel / download on three streams, double-buffered"}
         status = npa.npa_device_status(stream)
@@ -588,11 +602,8 @@ def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> Non
     clk = clocks.stop()
     kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     timed_ms = sum(kernel_ms) if flush is not None else t0.elapsed_time(t1)
-    if world > 1:
-        t = torch.tensor([timed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        timed_ms = float(t.item())
-    value = world * nbytes * args.steps / (timed_ms * 1e-3) / 1e9
+    timed_ms = max_over_ranks(timed_ms, world, dev)
+    value = whole_job_rate(world, nbytes, args.steps, timed_ms) / 1e9
     avg_ms = sum(kernel_ms) / args.steps
 
     e2e = None

@@ -1,11 +1,14 @@
 """bench.py's launcher contract on the CPU: the reference arm (the oracle on
 the host cores) under torchrun with two ranks prints exactly one JSON line
-from rank 0 and every rank exits 0."""
+from rank 0 and every rank exits 0; the replicas' timing reduction (slowest
+rank, whole-job rate) agrees on every rank under gloo."""
 import json
 import os
 import socket
 import subprocess
 import sys
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -28,3 +31,31 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["impl"] == "reference" and d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
     assert d["config"]["workload"] == "tiny_npa" and d["n_gpus"] == 2
+
+
+def _rank_timing(rank, world, port, out):
+    import torch.distributed as dist
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        ms = [12.5, 20.0, 7.25][rank]
+        slowest = bench.max_over_ranks(ms, world, "cpu")
+        with open(f"{out}.{rank}", "w") as f:
+            f.write(repr((slowest, bench.whole_job_rate(world, 1e12, 10, slowest))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_max_over_ranks_and_whole_job_rate_gloo(tmp_path, world):
+    """The multi-GPU bench (one replica per rank) reports the slowest rank's
+    time and the whole job's units over it; every rank must agree."""
+    import torch.multiprocessing as mp
+    out = str(tmp_path / "r")
+    mp.start_processes(_rank_timing, args=(world, _port(), out), nprocs=world, start_method="spawn")
+    import ast
+    results = [ast.literal_eval(open(f"{out}.{r}").read()) for r in range(world)]
+    slowest = max([12.5, 20.0, 7.25][:world])
+    for got_ms, rate in results:
+        assert got_ms == slowest
+        assert rate == world * 1e12 * 10 / (slowest * 1e-3)
