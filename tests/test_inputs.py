@@ -61,3 +61,22 @@ def test_smoothed_k_has_smaller_spread():
     w = PRESETS["npa_sdxl_2048"].replace(B=1, heads=1, H=32, W=32)
     k = bf16_bits_to_f64(make_inputs(w)["k"])
     assert 0.25 < k.std() < 0.45
+
+
+def test_later_row_inputs_follow_the_seed_recipe():
+    """Stale-row PCPP adds the previous step's k, v (seeds +5, +6); the
+    global-query form adds the global tokens' queries (seed +7). Each is an
+    independent N(0, 1) draw rounded to bf16, like q, k and v."""
+    from workloads import COMPARATORS
+    w = COMPARATORS["pcpp_stale_4x32_p0.3"].replace(B=1, heads=1, H=8, W=8, n_strips=2)
+    inp = make_inputs(w)
+    shape = (1, 1, 64, w.d)
+    for name, off in (("ks", 5), ("vs", 6)):
+        expect = f64_to_bf16_bits(np.random.default_rng(w.seed + off).standard_normal(shape))
+        np.testing.assert_array_equal(inp[name], expect)
+    assert not np.array_equal(inp["ks"], inp["k"])
+    g = COMPARATORS["gq_flux_4096"].replace(heads=2, H=4, W=4, G=10)
+    ginp = make_inputs(g)
+    expect = f64_to_bf16_bits(np.random.default_rng(g.seed + 7).standard_normal((1, 2, 10, g.d)))
+    np.testing.assert_array_equal(ginp["gq"], expect)
+    assert set(ginp) == {"q", "k", "v", "gk", "gv", "gq"}
