@@ -156,3 +156,24 @@ def test_query_subset_matches_full():
     qs = np.array([(1, 0, 0), (0, 1, 77), (1, 1, H * W - 1)], dtype=np.int32)
     sub = oracle.multidiffusion_attention(q, k, v, B=B, heads=h, H=H, W=W, d=d, patch=P, margin=m, queries=qs)
     np.testing.assert_array_equal(sub, full[qs[:, 0], qs[:, 1], qs[:, 2]])
+
+
+@pytest.mark.parametrize("dm", [-1, 1])
+def test_negative_control_margin_off_by_one(dm):
+    """A mistake planted in the oracle's arguments (margin off by one) must
+    break the hand-enumerated windows, the coverage counts and the pair
+    count, so the pins above would catch it."""
+    case = GOLDEN["cases"][0]
+    H, W, P, m = case["H"], case["W"], case["patch"], case["margin"] + dm
+    windows_ok = all(oracle.md_window_keys(H, W, P, m, *map(int, key.split(","))).tolist() == toks
+                     for key, toks in case["windows"].items())
+    counts_ok = all(oracle.md_window_count(H, W, P, m, int(t)) == c for t, c in case["counts"].items())
+    assert not windows_ok and not counts_ok
+    assert oracle.md_pair_count(H, W, P, m, 0) != case["pairs_G0"]
+
+
+def test_negative_control_patch_off_by_one():
+    case = GOLDEN["cases"][1]
+    H, W, P, m = case["H"], case["W"], case["patch"] + 1, case["margin"]
+    assert oracle.md_pair_count(H, W, P, m, 0) != case["pairs_G0"]
+    assert any(oracle.md_window_count(H, W, P, m, int(t)) != c for t, c in case["counts"].items())
