@@ -62,3 +62,15 @@ def test_shapes_checked(tensors):
         oracle.asg_guidance_combine(eps, ref[:, :, :-1], m, 1.0)
     with pytest.raises(ValueError):
         oracle.asg_guidance_combine(eps, ref, m[:, :, :-1], 1.0)
+
+
+def test_negative_controls_break_the_worked_example():
+    """Mistakes planted through the oracle's arguments - a sign error
+    (negated weight) or a complemented mask - must fail the hand-worked
+    example, so the pin catches them."""
+    g = GOLDEN
+    eps, ref, m = (f64_to_bf16_bits(np.array(g[k], dtype=np.float64)) for k in ("eps", "eps_ref", "mask"))
+    want = np.array(g["out"])
+    assert not np.array_equal(oracle.asg_guidance_combine(eps, ref, m, -g["w_t"]), want)
+    one_minus = f64_to_bf16_bits(1.0 - np.array(g["mask"], dtype=np.float64))
+    assert not np.array_equal(oracle.asg_guidance_combine(eps, ref, one_minus, g["w_t"]), want)
