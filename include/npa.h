@@ -25,6 +25,11 @@
  *  - Either geometry may append G global tokens (for example joint text
  *    tokens) to every key/value set. Global tokens produce no output rows.
  *
+ * Around these it provides the stale-row form of PCPP that runs across
+ * devices, the text-query half of joint attention (global tokens as queries),
+ * the overlapping-window attention NPA is compared with, and the ASG guidance
+ * combine; each declaration below cites its passage.
+ *
  * Arithmetic: bfloat16 inputs, float32 accumulation of Q.K^T and P.V on the
  * tensor cores, float32 online softmax with scale 1/sqrt(d), bfloat16 output
  * rounded to nearest even. Softmax probabilities are rounded to bfloat16
@@ -40,9 +45,9 @@
  * entry points allocate no device memory; the library's device state is one
  * status word per device (see npa_device_status) and the fixed scratch array
  * of npa_global_query_attention_fwd_noalloc. Host-side state is
- * limited to per-device capability checks and kernel attributes, set up under
- * a lock on first use, so the entry points are safe to call from several host
- * threads.
+ * limited to per-device capability checks, kernel attributes and that array's
+ * device address, set up under a lock on first use, so the entry points are
+ * safe to call from several host threads.
  *
  * CUDA graphs: after a first call on a device (which checks the device and
  * sets kernel attributes), npa_attention_fwd, pcpp_attention_fwd,
