@@ -38,6 +38,11 @@
  *  - Both geometries may append G global tokens (separate K/V tensors) to
  *    every key set, once each.
  *
+ * The same steps serve the later forms, each defined where it is written:
+ * PCPP with the borrowed rows read from the previous step's keys/values, the
+ * global tokens as queries over all keys, and the overlapping-window
+ * (MultiDiffusion-style) attention NPA is compared with.
+ *
  * Layout: q, k, v, out are [B, heads, H*W, d] with token t = row*W + col;
  * global k/v are [B, heads, G, d]. Inputs are bfloat16 bit patterns
  * (uint16); the output is double.
