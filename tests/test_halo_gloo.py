@@ -1,4 +1,5 @@
-"""Multi-rank PCPP on the CPU (gloo, world size 2 and 3): each rank owns a
+"""Multi-rank PCPP on the CPU (gloo, world size 2 to 4, even and uneven
+strip shares): each rank owns a
 range of strips, exchanges its boundary rows with its neighbours, and runs the
 two-source oracle for its strips. Exchanging the current step's rows and
 using them at once is the synchronous limit, so the ranks' outputs must equal
@@ -54,6 +55,8 @@ def _worker(rank, world, port, w, out_path):
     (2, Workload("halo_2", "pcpp", B=1, heads=2, H=16, W=6, d=16, n_strips=4, p=0.5)),
     (3, Workload("halo_3", "pcpp", B=2, heads=1, H=18, W=5, d=16, n_strips=6, p=0.4)),
     (2, Workload("halo_p1", "pcpp", B=1, heads=1, H=12, W=4, d=16, n_strips=2, p=1.0)),
+    # uneven share: 6 strips over 4 ranks hold 2, 2, 1, 1 strips
+    (4, Workload("halo_uneven", "pcpp", B=1, heads=2, H=24, W=4, d=16, n_strips=6, p=0.5)),
 ], ids=lambda x: x if isinstance(x, int) else x.name)
 def test_exchange_then_attend_equals_synchronous_pcpp(tmp_path, world, w):
     oracle.lib()  # build before the workers start
