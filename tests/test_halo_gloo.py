@@ -1,9 +1,9 @@
 """Multi-rank PCPP on the CPU (gloo, world size 2 to 4, even and uneven
-strip shares): each rank owns a
-range of strips, exchanges its boundary rows with its neighbours, and runs the
-two-source oracle for its strips. Exchanging the current step's rows and
-using them at once is the synchronous limit, so the ranks' outputs must equal
-the single-process single-source PCPP oracle exactly."""
+strip shares): each rank owns a range of strips, exchanges its boundary rows
+with its neighbours, and runs the two-source oracle for its strips.
+Exchanging the current step's rows and using them at once is the synchronous
+limit, so the ranks' outputs must equal the single-process single-source PCPP
+oracle exactly."""
 import socket
 
 import numpy as np
