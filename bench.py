@@ -630,8 +630,8 @@ def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> Non
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a.elapsed_time(b)
-        e2e = {"value": world * nbytes * args.steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+        e2e = {"value": whole_job_rate(world, nbytes, args.steps, e_ms) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}
     if rank != 0:
         return
