@@ -592,6 +592,9 @@ def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> Non
     clocks.start()
     time.sleep(0.3)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
     t0.record(stream)
     for i in range(args.steps):
         if flush is not None:
@@ -601,6 +604,8 @@ def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> Non
         ends[i].record(stream)
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
     clk = clocks.stop()
     kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     timed_ms = sum(kernel_ms) if flush is not None else t0.elapsed_time(t1)
