@@ -24,16 +24,6 @@ using npa::FwdParams;
 // below a millisecond).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
-// Query tiles per CTA for image-token queries at d = 64: 2 (128-key blocks)
-// or, built with NPA_D64_TILES=3, three tiles on 64-key blocks (three softmax
-// warpgroups share the exponential unit; measured no faster). d = 128 and the
-// global-token queries always run two tiles on 128-key blocks.
-#ifndef NPA_D64_TILES
-#define NPA_D64_TILES 2
-#endif
-static_assert(NPA_D64_TILES == 2 || NPA_D64_TILES == 3, "NPA_D64_TILES");
-constexpr int kD64Tiles = NPA_D64_TILES;
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -79,11 +69,7 @@ npa_status ensure_ready(int *sm_count = nullptr) {
             return NPA_ERR_CUDA;
         if (major != 10 || minor != 0) {
             ds.status = NPA_ERR_UNSUPPORTED;
-        } else if (
-#if NPA_D64_TILES == 3
-                   !set_smem(npa::npa_fwd_kernel<64, 3, 64, false>, npa::KCfg<64, 3, 64>::kSmemBytes) ||
-#endif
-                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, false>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
+        } else if (!set_smem(npa::npa_fwd_kernel<64, 2, 128, false>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<128, 2, 128, false>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<64, 2, 128, false, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
                    !set_smem(npa::npa_fwd_kernel<128, 2, 128, false, true>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
@@ -253,7 +239,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     int sm_count = 0;
     npa_status st = ensure_ready(&sm_count);
     if (st != NPA_OK) return st;
-    const int nt = (d == 64 && !md_part) ? kD64Tiles : 2;
+    const int nt = 2;  // query tiles per work unit
 
     FwdParams prm;
     std::memset(&prm, 0, sizeof(prm));
@@ -279,7 +265,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
         prm.tiles_c = (g.Pw + prm.qc - 1) / prm.qc;
         prm.tiles_r = (g.Ph + prm.qr - 1) / prm.qr;
     }
-    prm.kb = nt == 3 ? 64 : 128;
+    prm.kb = 128;
     prm.tiles_per_unit = nt;
     prm.kc_log2 = choose_kc_log2(g, prm.kb);
     prm.kr = prm.kb >> prm.kc_log2;
@@ -331,12 +317,6 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
         kernel = (const void *)npa::npa_fwd_kernel<128, 2, 128, false, true>;
         threads = npa::KCfg<128, 2, 128>::kThreads;
         smem = npa::KCfg<128, 2, 128>::kSmemBytes;
-#if NPA_D64_TILES == 3
-    } else if (d == 64) {
-        kernel = (const void *)npa::npa_fwd_kernel<64, 3, 64, false>;
-        threads = npa::KCfg<64, 3, 64>::kThreads;
-        smem = npa::KCfg<64, 3, 64>::kSmemBytes;
-#endif
     } else if (d == 64) {
         kernel = (const void *)npa::npa_fwd_kernel<64, 2, 128, false>;
         threads = npa::KCfg<64, 2, 128>::kThreads;

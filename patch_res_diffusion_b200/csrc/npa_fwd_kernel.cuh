@@ -3,8 +3,7 @@
 //
 // A persistent CTA works through units of NT query tiles (128 queries each) of
 // one patch that share the patch's key/value window, streamed in blocks of KB
-// keys. Every path runs NT = 2, KB = 128; NT = 3, KB = 64 (three softmax
-// warpgroups at d = 64) is a build option of the host launcher.
+// keys. Every path runs NT = 2, KB = 128.
 // Warps (NT + 1 warpgroups):
 //   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes 0..127)
 //   control warp 0     TMA producer (Q once per unit, then K and V blocks
@@ -73,20 +72,18 @@ constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 template <int D, int NT, int KB>
 struct KCfg {
     static_assert(D == 64 || D == 128, "head dim");
-    static_assert(NT == 2 || NT == 3, "tiles per CTA");
-    static_assert(KB == 64 || KB == 128, "keys per block");
-    static_assert(D == 64 || (NT == 2 && KB == 128), "d = 128 runs two tiles of 128-key blocks");
+    static_assert(NT == 2 && KB == 128, "two query tiles per CTA, 128-key blocks");
     static constexpr int kChunks = D / 64;                 // 64-element (128-byte) column blocks
     static constexpr int kQChunkBytes = 128 * 128;         // 128 query rows x 128 bytes
     static constexpr int kQTileBytes = kChunks * kQChunkBytes;
     static constexpr int kKVChunkBytes = KB * 128;         // KB key rows x 128 bytes
     static constexpr int kKVTileBytes = kChunks * kKVChunkBytes;
-    static constexpr int kStages = D == 128 ? 2 : (KB == 64 ? 8 : 4);
+    static constexpr int kStages = D == 128 ? 2 : 4;
     static constexpr int kThreads = 128 * (NT + 1);
     static constexpr int kCtlWarp = 4 * NT;                // first warp of the control warpgroup
-    static constexpr uint32_t kRegsLaunch = NT == 2 ? 168 : 128;
-    static constexpr uint32_t kRegsSoftmax = NT == 2 ? 216 : 144;
-    static constexpr uint32_t kRegsCtl = NT == 2 ? 72 : 80;
+    static constexpr uint32_t kRegsLaunch = 168;
+    static constexpr uint32_t kRegsSoftmax = 216;
+    static constexpr uint32_t kRegsCtl = 72;
     static_assert(NT * 128 * kRegsSoftmax + 128 * kRegsCtl == kThreads * kRegsLaunch, "register split");
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = NT * kQTileBytes;
@@ -443,7 +440,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, uint64
     return __all_sync(0xffffffffu, got);
 }
 
-// Row maximum of 128 scores: eight independent chains of three-input maxima.
 // Maximum of a row's KB scores: eight interleaved chains of three-input maxima.
 template <int KB>
 __device__ __forceinline__ float row_max(const float (&s)[KB]) {
@@ -460,39 +456,6 @@ __device__ __forceinline__ float row_max(const float (&s)[KB]) {
     return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
 }
 
-// Fraction (in eighths) of the exponentials evaluated on the FMA pipe. Off
-// by default: measured on B200 at d = 64, every fraction from 1/8 to 5/8 made
-// the kernel slower (the exponential phase is limited by instruction issue
-// and latency as much as by the special-function unit's throughput).
-#ifndef NPA_EXP_EMU8
-#define NPA_EXP_EMU8 0
-#endif
-
-// 2^x for a pair of arguments without the special-function unit: Cody-Waite
-// reduction x = j + f, j = round(x) by the float32 magic-number addition
-// (1.5 * 2^23), f in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial
-// (relative error 7.5e-5, fitted by fit_exp2_poly.py); 2^j added to the
-// exponent field. Arguments below -125 (masked keys: -inf) give exactly 0.
-__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float &p0, float &p1) {
-    float x0, x1;
-    sm100::unpack_f32x2(x2, x0, x1);
-    const uint64_t xc = sm100::pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t magic = sm100::pack_f32x2(12582912.f, 12582912.f);
-    const uint64_t neg_magic = sm100::pack_f32x2(-12582912.f, -12582912.f);
-    const uint64_t t = sm100::add_f32x2(xc, magic);
-    const uint64_t jn = sm100::add_f32x2(neg_magic, t);                        // j
-    const uint64_t f = sm100::fma_f32x2(jn, sm100::pack_f32x2(-1.f, -1.f), xc);  // x - j
-    uint64_t p = sm100::fma_f32x2(sm100::pack_f32x2(0.0551716685295105f, 0.0551716685295105f), f,
-                                  sm100::pack_f32x2(0.2426111251115799f, 0.2426111251115799f));
-    p = sm100::fma_f32x2(p, f, sm100::pack_f32x2(0.6932609677314758f, 0.6932609677314758f));
-    p = sm100::fma_f32x2(p, f, sm100::pack_f32x2(0.9999280571937561f, 0.9999280571937561f));
-    float q0, q1, t0, t1;
-    sm100::unpack_f32x2(p, q0, q1);
-    sm100::unpack_f32x2(t, t0, t1);
-    p0 = x0 < -125.f ? 0.f : __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    p1 = x1 < -125.f ? 0.f : __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 // p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum returned.
 template <int KB>
 __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2]) {
@@ -503,15 +466,10 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
 #pragma unroll
     for (int i = 0; i < KB / 2; ++i) {
         const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
-        float p0, p1;
-        if ((i & 7) < NPA_EXP_EMU8) {
-            exp2_poly_x2(x2, p0, p1);
-        } else {
-            float x0, x1;
-            sm100::unpack_f32x2(x2, x0, x1);
-            p0 = sm100::ex2_approx(x0);
-            p1 = sm100::ex2_approx(x1);
-        }
+        float x0, x1;
+        sm100::unpack_f32x2(x2, x0, x1);
+        const float p0 = sm100::ex2_approx(x0);
+        const float p1 = sm100::ex2_approx(x1);
         pk[i] = sm100::pack_bf16x2(p0, p1);
         acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
     }
@@ -562,10 +520,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         float s[KB];
         {
             uint32_t sr[KB];
-            if constexpr (KB == 128)
-                sm100::tmem_ld128(tS, sr);
-            else
-                sm100::tmem_ld64(tS, sr);
+            sm100::tmem_ld128(tS, sr);
 #pragma unroll
             for (int i = 0; i < KB; ++i) s[i] = __uint_as_float(sr[i]);
         }
@@ -640,10 +595,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
         }
         l = l * alpha + blk_sum;
-        if constexpr (KB == 128)
-            sm100::tmem_st64(tP, pk);
-        else
-            sm100::tmem_st32(tP, pk);
+        sm100::tmem_st64(tP, pk);
         sm100::tc_fence_before();
         sm100::mbar_arrive(&bars[C::bPFull + q]);
         R_prev = R;

@@ -32,16 +32,14 @@ def run(exe, *args):
 # BH, H, W, Ph, Pw, mh, mw, kb, kc_log2, tiles_per_unit, n_qblocks, patch_begin, patch_count
 CASES = {
     "npa_sdxl_4096": (20, 256, 256, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
-    "npa_sdxl_4096_triples": (20, 256, 256, 64, 64, 32, 32, 64, 5, 3, 11, 0, -1),  # NPA_D64_TILES=3
     "npa_flux_4096": (24, 256, 256, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
     "npa_sdxl_2048": (20, 128, 128, 64, 64, 32, 32, 128, 5, 2, 16, 0, -1),
-    "ragged": (3, 40, 37, 16, 16, 5, 5, 64, 4, 3, 1, 0, -1),
+    "ragged": (3, 40, 37, 16, 16, 5, 5, 128, 4, 2, 1, 0, -1),
     "ragged_small_patches": (2, 100, 100, 9, 9, 3, 3, 128, 3, 2, 1, 0, -1),
     "pcpp_4x32": (20, 128, 128, 32, 128, 10, 0, 128, 7, 2, 16, 0, -1),
     "pcpp_8x16": (20, 128, 128, 16, 128, 13, 0, 128, 7, 2, 8, 0, -1),
-    "pcpp_8x16_triples": (20, 128, 128, 16, 128, 13, 0, 64, 6, 3, 6, 0, -1),
     "pcpp_strip_range": (4, 64, 64, 8, 64, 3, 0, 128, 6, 2, 2, 3, 4),
-    "npa_patch_range": (4, 64, 64, 16, 16, 4, 4, 64, 4, 3, 1, 3, 7),
+    "npa_patch_range": (4, 64, 64, 16, 16, 4, 4, 128, 4, 2, 1, 3, 7),
     "unordered": (2, 61, 59, 3, 4, 1, 2, 128, 3, 2, 1, 0, -1),        # 315 patches: natural order
     "fifteen_classes": (2, 300, 300, 20, 20, 60, 60, 128, 3, 2, 1, 0, -1),
     "too_many_classes": (2, 300, 300, 20, 20, 100, 100, 128, 3, 2, 1, 0, -1),  # ordered, no class table
@@ -64,9 +62,6 @@ def test_concurrent_units_share_heads(checker):
     r = run(checker, *CASES["npa_sdxl_4096"], 148)
     assert r["classes"] == 3
     assert r["wave_heads"] <= 3
-    r = run(checker, *CASES["npa_sdxl_4096_triples"], 148)
-    assert r["classes"] == 3
-    assert r["wave_heads"] <= 5
 
 
 def test_fallbacks(checker):
