@@ -629,12 +629,16 @@ def run_asg(args, w: AsgWorkload, rank: int, world: int, local_rank: int) -> Non
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(args.steps):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
         e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
         e2e = {"value": whole_job_rate(world, nbytes, args.steps, e_ms) / 1e9, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / args.steps}

@@ -156,7 +156,12 @@ npa_status npa_global_query_attention_fwd(const void *gq, const void *k, const v
  * until the process exits); nothing is allocated per call. The array must
  * hold at least two partial results, 2 * B * heads * G * (d + 2) * 4 bytes
  * <= 16 MiB, else the call returns NPA_ERR_UNSUPPORTED before touching the
- * device; the split count is also limited by the array. The
+ * device. This is stricter than npa_global_query_attention_fwd, which runs
+ * such a problem unsplit when its workspace is too small: a caller of the
+ * fixed array learns its limit from the status instead of getting a call
+ * that silently loses the split's parallelism. The split count is also
+ * limited by the array (FLUX's 24 heads x 512 text tokens at d = 128 run
+ * with 2 splits). The
  * first call on each device looks up the array's device address (with that
  * device current) and should come before any stream capture. Every call
  * shares the array and overwrites it; nothing in it needs to start at zero.
@@ -217,14 +222,27 @@ npa_status asg_guidance_combine(const void *eps, const void *eps_ref, const void
  * count on the current device (0: no split needed, or invalid arguments). */
 size_t npa_global_query_workspace_size(int B, int heads, int H, int W, int d, int G);
 
-/* r = ceil(p * strip_rows) (double, 1e-9 allowance), limited to
+/* Rows a strip borrows from each adjacent strip (PCPP review, "What carries
+ * the argument": p is the fraction of each neighbour patch's height that is
+ * concatenated into the local key/value set; "Core claim": the top or bottom
+ * p-fraction). The pages do not say how p * strip_rows is rounded; the reading
+ * taken is r = ceil(p * strip_rows - 1e-9) in double, so that a product that
+ * is an integer up to rounding (0.3 * 10) is not rounded up, limited to
  * [0, strip_rows]. Returns -1 if strip_rows < 1 or p is outside [0, 1]. */
 int pcpp_neighbor_rows(int strip_rows, double p);
 
-/* Useful floating-point work of one call: 4 * d * B * heads * (sum over
- * queries of the key-set size, global keys included) - two multiply-adds per
- * (query, key, channel) for Q.K^T and P.V; softmax work not counted.
- * Returns a negative value for invalid geometry arguments. */
+/* Useful floating-point work of one call, the numerator of the library's
+ * throughput figure: 4 * d * B * heads * (sum over queries of the key-set
+ * size, global keys included), i.e. two multiply-adds per (query, key,
+ * channel), one for Q.K^T and one for P.V; softmax work is not counted. It
+ * counts only the entries of the restricted attention matrix - the work that
+ * remains once the key set is restricted (ScaleDiff summary, "Approach": the
+ * neighbourhood restriction keeps the self-attention cost from growing with
+ * overlapping patches; PCPP review, "What carries the argument": partial
+ * conditioning shrinks the attention matrix) - not the full-attention work
+ * avoided. Key-set sizes follow the geometry of npa_attention_fwd and
+ * pcpp_attention_fwd. Returns a negative value for invalid geometry
+ * arguments. */
 double npa_useful_flops(int B, int heads, int H, int W, int d, int patch, int margin, int G);
 double pcpp_useful_flops(int B, int heads, int H, int W, int d, int n_strips, double p, int G);
 
