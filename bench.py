@@ -53,6 +53,8 @@ def parse():
                     help="approximate CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip timing the other target workloads (per_config) after the headline one")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write 256 MB between launches even when the inputs exceed L2 (cold-cache variant)")
     return ap.parse_args()
@@ -265,23 +267,44 @@ def useful_flops_host(w: Workload) -> float:
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """Samples SM clocks, power and throttle reasons with nvidia-smi every
+    20 ms; ``stop()`` keeps the samples stamped inside the window between
+    ``mark_begin()`` and ``mark_end()`` (host wall clock; the timed region),
+    or the nearest sample when none falls inside."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join("/tmp", f"npa_clocks_{os.getpid()}.csv")
+        self.path = os.path.join("/tmp", f"npa_clocks_{os.getpid()}_{device_index}.csv")
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    @staticmethod
+    def _stamp(text: str):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(text, fmt).timestamp()
+            except ValueError:
+                continue
+        return None
 
     def stop(self):
         if self.proc is None:
@@ -296,41 +319,55 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    rows.append({"sm": float(parts[1]), "max": float(parts[2]), "power": float(parts[3]),
-                                 "hw": parts[5], "hw_thermal": parts[6], "sw_thermal": parts[7],
-                                 "sw_power": parts[8]})
+                    rows.append({"t": self._stamp(parts[0]), "sm": float(parts[2]), "max": float(parts[3]),
+                                 "power": float(parts[4]), "hw": parts[6], "hw_thermal": parts[7],
+                                 "sw_thermal": parts[8], "sw_power": parts[9]})
                 except ValueError:
                     continue
         os.unlink(self.path)
         if not rows:
             return None
-        loaded = [r for r in rows if r["power"] > 300.0] or rows
+        inside = [r for r in rows if r["t"] is not None and self.t0 is not None and self.t1 is not None
+                  and self.t0 <= r["t"] <= self.t1]
+        basis = "samples stamped inside the timed region"
+        if not inside:
+            mid = 0.5 * (self.t0 + self.t1) if self.t0 is not None and self.t1 is not None else None
+            stamped = [r for r in rows if r["t"] is not None]
+            if mid is not None and stamped:
+                inside = [min(stamped, key=lambda r: abs(r["t"] - mid))]
+                basis = "no sample inside the timed region; the nearest one"
+            else:
+                inside = rows
+                basis = "no timestamps; every sample"
         reasons = set()
-        for r in loaded:
+        for r in inside:
             for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
                               ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
                 if r[key].lower().startswith("active"):
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["max"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(loaded),
-                "power_w_max": max(r["power"] for r in rows)}
+        return {"sm_mhz": statistics.median(r["sm"] for r in inside), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(inside), "basis": basis,
+                "power_w_max": max(r["power"] for r in inside),
+                "region_s": (self.t1 - self.t0) if self.t0 is not None and self.t1 is not None else None}
 
 
 # ---------------------------------------------------------------------------
 # The GPU arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
+def prepare(w: Workload, dev, flush_l2: bool, inp: dict = None):
+    """Device tensors, workspaces and the library call of one workload step.
+    Returns a namespace with ``call()`` (one step on the current stream),
+    the tensors, the useful flops, the minimum HBM bytes and the L2 flush
+    buffer (allocated when the inputs fit in twice the L2 or when asked)."""
+    import types
     import torch
-    import torch.distributed as dist
     import patch_res_diffusion_b200 as npa
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    inp = make_inputs(w)
+    inp = make_inputs(w) if inp is None else inp
 
     def dev_bf16(a):
         return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -343,7 +380,6 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     gq = dev_bf16(inp["gq"]) if w.geometry == "gq" else None
     o = torch.empty_like(gq if gq is not None else q)
     stream = torch.cuda.current_stream(dev)
-    flops = useful_flops(w)
     # minimum HBM bytes of one call: every input read once, the output written once
     bytes_io = (q.numel() * 4 + (2 * gk.numel() if w.G else 0)) * 2  # q, k, v, o (+ global k, v)
     if w.geometry == "gq":  # global queries and output, global k, v, image k, v
@@ -351,7 +387,7 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     elif w.geometry == "pcpp_stale":  # + the borrowed rows of the previous step's k, v
         r = npa.pcpp_neighbor_rows(w.H // w.n_strips, w.p)
         bytes_io += 2 * (2 * r * (w.n_strips - 1)) * w.W * w.d * 2 * w.B * w.heads
-    needs_flush = bytes_io < 2 * L2_BYTES or args.flush_l2
+    needs_flush = bytes_io < 2 * L2_BYTES or flush_l2
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if needs_flush else None
 
     md_bytes = npa.npa_multidiffusion_workspace_size(w.B, w.heads, w.H, w.W, w.d, w.patch, w.margin) \
@@ -375,16 +411,33 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         else:
             npa.pcpp_attention_fwd(q, k, v, o, w.B, w.heads, w.H, w.W, w.d, w.n_strips, w.p, gk, gv, w.G, stream)
 
-    for _ in range(args.warmup):
+    launches = 2 if w.geometry == "md" or gq_bytes > 0 else 1
+    return types.SimpleNamespace(w=w, inp=inp, q=q, k=k, v=v, gk=gk, gv=gv, gq=gq, o=o, stream=stream,
+                                 flops=useful_flops(w), bytes_io=bytes_io, flush=flush, md_ws=md_ws,
+                                 md_bytes=md_bytes, call=call, launches=launches)
+
+
+def timed_steps(prep, steps: int, warmup: int, dev, world: int, local_rank: int) -> dict:
+    """``warmup`` untimed steps, then exactly ``steps`` timed ones bracketed by
+    a synchronize (and a barrier when world > 1) on both sides, with CUDA
+    events around every step and around the region on the launching stream.
+    With a flush buffer, 256 MB are written before every step (outside the
+    per-step events) and the region's time is the sum of the per-step
+    times. Clocks are sampled during the region."""
+    import torch
+    import torch.distributed as dist
+    import patch_res_diffusion_b200 as npa
+
+    stream, flush, call = prep.stream, prep.flush, prep.call
+    for _ in range(warmup):
         if flush is not None:
             flush.fill_(1)
         call()
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local_rank)
@@ -393,8 +446,9 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
+    clocks.mark_begin()
     t_begin.record(stream)
-    for i in range(args.steps):
+    for i in range(steps):
         if flush is not None:
             flush.fill_(1)
         starts[i].record(stream)
@@ -402,18 +456,57 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         ends[i].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark_end()
     if world > 1:
         dist.barrier()
+    time.sleep(0.1)
     clk = clocks.stop()
     status = npa.npa_device_status(stream)
     if status != npa.NPA_OK:
         raise RuntimeError(f"device status {npa.npa_status_string(status)}")
-
-    kernel_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    kernel_ms_sum = sum(kernel_ms)
+    kernel_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     elapsed_ms = t_begin.elapsed_time(t_end)
-    timed_ms = kernel_ms_sum if flush is not None else elapsed_ms
-    timed_ms = max_over_ranks(timed_ms, world, dev)
+    return {"kernel_ms": kernel_ms, "timed_ms": sum(kernel_ms) if flush is not None else elapsed_ms,
+            "clocks": clk}
+
+
+def per_config_entry(prep, res: dict, pk: dict) -> dict:
+    """One workload's figures for the ``per_config`` object of the line."""
+    km = res["kernel_ms"]
+    avg = sum(km) / len(km)
+    tf = prep.flops / (avg * 1e-3) / 1e12
+    return {
+        "config": describe(prep.w),
+        "ms": {"median": statistics.median(km), "best": min(km), "mean": avg},
+        "useful_tflops": tf,
+        "frac_of_burst": tf / pk["bf16_tflops"],
+        "frac_of_sustained": tf / pk["bf16_tflops_sustained"],
+        "useful_flops_per_call": prep.flops,
+        "l2": "flushed (256 MB write) before every launch" if prep.flush is not None else "inputs larger than L2",
+        "launches_per_call": prep.launches,
+        "steps": len(km),
+        "clocks": res["clocks"],
+    }
+
+
+# The other target workloads reported beside the headline one.
+PER_CONFIG = ["tiny_npa", "pcpp_4x32_p0.3", "pcpp_8x16_p0.8", "npa_sdxl_2048", "npa_flux_4096"]
+
+
+def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
+    import torch
+    import torch.distributed as dist
+    import patch_res_diffusion_b200 as npa
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    prep = prepare(w, dev, args.flush_l2)
+    inp, q, k, v, gk, gv, o, stream = prep.inp, prep.q, prep.k, prep.v, prep.gk, prep.gv, prep.o, prep.stream
+    flops, bytes_io, flush, md_ws, md_bytes = prep.flops, prep.bytes_io, prep.flush, prep.md_ws, prep.md_bytes
+    res = timed_steps(prep, args.steps, args.warmup, dev, world, local_rank)
+    kernel_ms, clk = res["kernel_ms"], res["clocks"]
+    kernel_ms_sum = sum(kernel_ms)
+    timed_ms = max_over_ranks(res["timed_ms"], world, dev)
     value = whole_job_rate(world, flops, args.steps, timed_ms) / 1e12
     avg_kernel_ms = kernel_ms_sum / args.steps
 
@@ -487,6 +580,19 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         if status != npa.NPA_OK:
             raise RuntimeError(f"device status {npa.npa_status_string(status)}")
 
+    # The other target workloads, timed the same way on this GPU (one process,
+    # N = 1 only; the headline line stays on the requested workload).
+    per_config = None
+    if world == 1 and not args.no_per_config and w.name == DEFAULT_WORKLOAD:
+        pk, _ = peaks()
+        per_config = {}
+        for name in PER_CONFIG:
+            other = prepare(PRESETS[name], dev, args.flush_l2)
+            per_config[name] = per_config_entry(other, timed_steps(other, args.steps, args.warmup, dev, 1,
+                                                                   local_rank), pk)
+            del other
+            torch.cuda.empty_cache()
+
     if rank != 0:
         return
     pk, pk_kind = peaks()
@@ -529,9 +635,11 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk,
-        "gpu_launches": args.steps * (2 if w.geometry == "md" or gq_bytes > 0 else 1),
+        "gpu_launches": args.steps * prep.launches,
         "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
     }
+    if per_config is not None:
+        line["per_config"] = per_config
     print(json.dumps(line), flush=True)
 
 

@@ -1,5 +1,5 @@
 """Helpers shared by the GPU parity tests: device transfer, the comparison
-gates and the query sampler used at full workload sizes."""
+gates and the query sets used at full workload sizes."""
 from __future__ import annotations
 
 import numpy as np
@@ -100,3 +100,34 @@ def sample_queries(w: Workload, n_random: int = 512, seed: int = 0, max_bh: int 
     for _ in range(n_random):
         out.append((int(rng.integers(w.B)), int(rng.integers(w.heads)), int(rng.integers(N))))
     return np.array(out, dtype=np.int32)
+
+
+def patch_edge_queries(w: Workload, random_frac: float = 0.01, seed: int = 0) -> np.ndarray:
+    """Query set for the workloads too large for a full oracle run: for every
+    (b, h) and every patch, the patch's first 128 and last 128 queries in
+    row-major order within the patch (its first and last query tile), plus
+    ``random_frac`` of all (b, h, t) rows drawn uniformly without
+    replacement. Returns an (n, 3) int32 array of (b, h, t), unique rows."""
+    rng = np.random.default_rng(seed)
+    N = w.H * w.W
+    per_patch = []
+    for r0 in range(0, w.H, w.patch):
+        for c0 in range(0, w.W, w.patch):
+            rows = np.arange(r0, min(w.H, r0 + w.patch))
+            cols = np.arange(c0, min(w.W, c0 + w.patch))
+            toks = (rows[:, None] * w.W + cols[None, :]).ravel()   # row-major within the patch
+            per_patch.append(np.unique(np.concatenate([toks[:128], toks[-128:]])))
+    toks = np.concatenate(per_patch)
+    bh = np.arange(w.B * w.heads)
+    flat = (bh[:, None].astype(np.int64) * N + toks[None, :]).ravel()
+    n_rand = int(np.ceil(random_frac * w.B * w.heads * N))
+    flat = np.unique(np.concatenate([flat, rng.choice(w.B * w.heads * N, size=n_rand, replace=False)]))
+    return np.stack([flat // (w.heads * N), (flat // N) % w.heads, flat % N], axis=1).astype(np.int32)
+
+
+def gather_rows(o, w: Workload, qs: np.ndarray) -> np.ndarray:
+    """Rows (b, h, t) of a device output [B, heads, N, d], as float64."""
+    import torch
+    flat = o.reshape(w.B * w.heads * w.H * w.W, w.d)
+    idx = torch.from_numpy((qs[:, 0].astype(np.int64) * w.heads + qs[:, 1]) * (w.H * w.W) + qs[:, 2])
+    return to_f64(flat.index_select(0, idx.to(o.device)))

@@ -52,24 +52,22 @@ def test_global_query_full_parity(B, heads, H, W, d, G, split):
     assert passes(m), m
 
 
+_FLUX_REF = {}
+
+
 @pytest.mark.parametrize("split", [False, True])
-def test_global_query_flux_shape_sampled(split):
+def test_global_query_flux_shape_every_row(split):
     """FLUX-like 4096^2 joint attention, text half: 512 text queries x
-    (65,536 image + 512 text) keys, 24 heads, d = 128."""
+    (65,536 image + 512 text) keys, 24 heads, d = 128, every output row."""
     import patch_res_diffusion_b200 as npa
     B, heads, H, W, d, G = 1, 24, 256, 256, 128, 512
     inp = make(B, heads, H, W, d, G, 5)
     if split:
         assert npa.npa_global_query_workspace_size(B, heads, H, W, d, G) > 0
-    o = gpu(inp, H, W, split)
-    torch.cuda.synchronize()
-    rng = np.random.default_rng(1)
-    qs = np.stack([np.zeros(96, dtype=np.int32), rng.integers(heads, size=96), rng.integers(G, size=96)], 1)
-    qs = np.concatenate([qs, [[0, 0, 0], [0, 23, 511], [0, 11, 255]]]).astype(np.int32)
-    ref = oracle.global_query_attention(inp["gq"], inp["k"], inp["v"], inp["gk"], inp["gv"], B=B, heads=heads,
-                                        H=H, W=W, d=d, G=G, queries=qs)
-    got = to_f64(o[qs[:, 0], qs[:, 1], qs[:, 2]])
-    m = compare(got, ref)
-    log_metrics(f"global query FLUX split={split} (sampled)", m)
+    got = to_f64(gpu(inp, H, W, split))
+    if "ref" not in _FLUX_REF:
+        _FLUX_REF["ref"] = oracle.global_query_attention(inp["gq"], inp["k"], inp["v"], inp["gk"], inp["gv"], B=B,
+                                                         heads=heads, H=H, W=W, d=d, G=G)
+    m = compare(got, _FLUX_REF["ref"])
+    log_metrics(f"global query FLUX split={split} (every row)", m)
     assert passes(m), m
-    assert bool(torch.isfinite(o).all())
