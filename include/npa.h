@@ -83,7 +83,8 @@ typedef enum {
     NPA_ERR_UNSUPPORTED = 2,     /* d not in {64,128}, size beyond limits, device not sm_100 */
     NPA_ERR_MISALIGNED = 3,      /* a pointer is not 16-byte aligned */
     NPA_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
-    NPA_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait ran out */
+    NPA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out */
+    NPA_ERR_DEVICE_BOUNDS = 6    /* bounds-checking build only: a device-side bounds check failed */
 } npa_status;
 
 /* Optional global tokens appended to every key/value set.
@@ -256,6 +257,27 @@ npa_status npa_device_status(npa_stream_t stream);
  * expected outcome is that npa_device_status() then returns
  * NPA_ERR_DEVICE_TIMEOUT. Returns NPA_ERR_INVALID_ARG for a bad limit. */
 npa_status npa_selftest_wait_timeout(uint32_t limit_us, npa_stream_t stream);
+
+/* Bounds-checking build (libnpa_b200_debug.so, compiled with
+ * NPA_DEBUG_BOUNDS; the pages have no counterpart, this is a debugging aid
+ * standing in for a memory checker). Every kernel checks each TMA box origin
+ * against its tensor's extent and each output row against the output's row
+ * count; a failed check records NPA_ERR_DEVICE_BOUNDS in the status word,
+ * clamps the load into the tensor or skips the store, and the kernel carries
+ * on. The normal library has no checks and does not export the function
+ * below.
+ *
+ * npa_debug_withhold_arrival_once: the next npa_attention_fwd,
+ * pcpp_attention_fwd, pcpp_attention_fwd_stale or
+ * npa_multidiffusion_attention_fwd launch runs with bounded waits of
+ * `wait_limit_us` microseconds (1..1000000), and its first CTA withholds the
+ * arrival that announces the second key block's P of its last query tile.
+ * That wait runs out, the CTA records NPA_ERR_DEVICE_TIMEOUT, stops issuing,
+ * waits for the copies and products already issued, frees its tensor memory
+ * and exits; the call's output is undefined. It exercises the kernel's abort
+ * path without faulting or hanging the GPU; the next call runs normally.
+ * Returns NPA_ERR_INVALID_ARG for a bad limit. */
+npa_status npa_debug_withhold_arrival_once(uint32_t wait_limit_us);
 
 /* Static, human-readable name of a status code. */
 const char *npa_status_string(npa_status status);

@@ -43,10 +43,12 @@ __all__ = [
     "pcpp_attention", "pcpp_attention_fwd_stale", "pcpp_attention_stale", "npa_global_query_attention_fwd",
     "npa_global_query_workspace_size", "npa_global_query_attention_fwd_noalloc", "global_query_attention",
     "npa_multidiffusion_attention_fwd", "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops",
-    "multidiffusion_attention", "asg_guidance_combine", "asg_combine", "EXPORTED_SYMBOLS",
+    "multidiffusion_attention", "asg_guidance_combine", "asg_combine", "EXPORTED_SYMBOLS", "DEBUG_LIB_PATH",
+    "DEBUG_ONLY_SYMBOLS", "NPA_ERR_DEVICE_BOUNDS", "use_bounds_checking", "npa_debug_withhold_arrival_once",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200.so")
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnpa_b200_debug.so")
 
 NPA_OK = 0
 NPA_ERR_INVALID_ARG = 1
@@ -54,6 +56,7 @@ NPA_ERR_UNSUPPORTED = 2
 NPA_ERR_MISALIGNED = 3
 NPA_ERR_CUDA = 4
 NPA_ERR_DEVICE_TIMEOUT = 5
+NPA_ERR_DEVICE_BOUNDS = 6
 
 EXPORTED_SYMBOLS = (
     "npa_attention_fwd", "pcpp_attention_fwd", "pcpp_attention_fwd_stale", "pcpp_neighbor_rows", "npa_useful_flops",
@@ -62,6 +65,8 @@ EXPORTED_SYMBOLS = (
     "npa_global_query_attention_fwd_noalloc", "npa_multidiffusion_attention_fwd",
     "npa_multidiffusion_workspace_size", "npa_multidiffusion_useful_flops", "asg_guidance_combine",
 )
+# exported by the bounds-checking build only
+DEBUG_ONLY_SYMBOLS = ("npa_debug_withhold_arrival_once",)
 
 
 class NpaError(RuntimeError):
@@ -75,15 +80,32 @@ class _GlobalKV(ctypes.Structure):
 
 
 _LIB: Optional[ctypes.CDLL] = None
+_LOADED = {}
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded C library. Raises if it has not been built."""
+    """The C library in use (the normal build unless use_bounds_checking(True)
+    switched to the bounds-checking one). Raises if it has not been built."""
     global _LIB
     if _LIB is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m patch_res_diffusion_b200.build`")
-        L = ctypes.CDLL(LIB_PATH)
+        _LIB = _load(LIB_PATH)
+    return _LIB
+
+
+def use_bounds_checking(on: bool) -> None:
+    """Routes every call of this module to the bounds-checking build
+    (``libnpa_b200_debug.so``: device-side checks of every TMA box origin and
+    output row, NPA_ERR_DEVICE_BOUNDS on a failure) or back to the normal one.
+    Each library keeps its own device status word."""
+    global _LIB
+    _LIB = _load(DEBUG_LIB_PATH if on else LIB_PATH)
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _LOADED:
+        if not os.path.exists(path):
+            raise ImportError(f"{path} is missing: build it with `python -m patch_res_diffusion_b200.build`")
+        L = ctypes.CDLL(path)
         vp, i, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
         gkv = ctypes.POINTER(_GlobalKV)
         L.npa_attention_fwd.argtypes = [vp, vp, vp, vp, i, i, i, i, i, i, i, gkv, vp]
@@ -119,8 +141,11 @@ def lib() -> ctypes.CDLL:
         L.npa_selftest_wait_timeout.restype = i
         L.npa_status_string.argtypes = [i]
         L.npa_status_string.restype = ctypes.c_char_p
-        _LIB = L
-    return _LIB
+        if path == DEBUG_LIB_PATH:
+            L.npa_debug_withhold_arrival_once.argtypes = [ctypes.c_uint32]
+            L.npa_debug_withhold_arrival_once.restype = i
+        _LOADED[path] = L
+    return _LOADED[path]
 
 
 def _ptr(x) -> Optional[int]:
@@ -250,6 +275,16 @@ def npa_device_status(stream=None) -> int:
 
 def npa_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check(lib().npa_selftest_wait_timeout(int(limit_us), _stream(stream)), "npa_selftest_wait_timeout")
+
+
+def npa_debug_withhold_arrival_once(wait_limit_us: int) -> None:
+    """C ``npa_debug_withhold_arrival_once`` (bounds-checking build only):
+    the next attention launch's first CTA withholds one arrival and its
+    bounded waits of ``wait_limit_us`` run out (the abort path)."""
+    L = lib()
+    if not hasattr(L, "npa_debug_withhold_arrival_once"):
+        raise NpaError(NPA_ERR_UNSUPPORTED, "npa_debug_withhold_arrival_once needs use_bounds_checking(True)")
+    _check(L.npa_debug_withhold_arrival_once(int(wait_limit_us)), "npa_debug_withhold_arrival_once")
 
 
 def npa_status_string(code: int) -> str:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -24,6 +25,12 @@ using npa::FwdParams;
 // below a millisecond).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+#ifdef NPA_DEBUG_BOUNDS
+// Bounds-checking build: wait limit (microseconds) of the next attention
+// launch whose CTA 0 withholds one arrival; 0 = none pending.
+std::atomic<unsigned> g_debug_stall_us{0};
+#endif
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -35,17 +42,27 @@ struct DeviceState {
     bool checked = false;
     npa_status status = NPA_ERR_UNSUPPORTED;
     int sm_count = 0;
+    int l2_bytes = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
-bool set_smem(void (*kernel)(FwdParams), int bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+// Sets an attention kernel's shared-memory limit and checks that it was
+// compiled with the register count its warp roles redistribute: the softmax
+// warpgroups' setmaxnreg.inc draws on the registers the block was launched
+// with, and would never complete if the launch held fewer.
+template <int D, bool GQ, bool MD = false>
+bool prepare_kernel() {
+    using C = npa::KCfg<D, 2, 128>;
+    void (*kernel)(FwdParams) = npa::npa_fwd_kernel<D, 2, 128, GQ, MD>;
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess || attr.numRegs != (int)C::kRegsLaunch) return false;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) == cudaSuccess;
 }
 
 // Resolves the tensor-map encoder and checks (once per device) that the
 // current device is an sm_100 part; sets the kernels' shared-memory limits.
 // On success *sm_count holds the device's multiprocessor count.
-npa_status ensure_ready(int *sm_count = nullptr) {
+npa_status ensure_ready(int *sm_count = nullptr, int *l2_bytes = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return NPA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return NPA_ERR_UNSUPPORTED;
@@ -65,23 +82,21 @@ npa_status ensure_ready(int *sm_count = nullptr) {
             cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
             return NPA_ERR_CUDA;
         if (cudaDeviceGetAttribute(&ds.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-            ds.sm_count < 1)
+            ds.sm_count < 1 || cudaDeviceGetAttribute(&ds.l2_bytes, cudaDevAttrL2CacheSize, dev) != cudaSuccess)
             return NPA_ERR_CUDA;
         if (major != 10 || minor != 0) {
             ds.status = NPA_ERR_UNSUPPORTED;
-        } else if (!set_smem(npa::npa_fwd_kernel<64, 2, 128, false>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
-                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, false>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
-                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, false, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
-                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, false, true>, npa::KCfg<128, 2, 128>::kSmemBytes) ||
-                   !set_smem(npa::npa_fwd_kernel<64, 2, 128, true>, npa::KCfg<64, 2, 128>::kSmemBytes) ||
-                   !set_smem(npa::npa_fwd_kernel<128, 2, 128, true>, npa::KCfg<128, 2, 128>::kSmemBytes)) {
-            return NPA_ERR_CUDA;
+        } else if (!prepare_kernel<64, false>() || !prepare_kernel<128, false>() ||
+                   !prepare_kernel<64, false, true>() || !prepare_kernel<128, false, true>() ||
+                   !prepare_kernel<64, true>() || !prepare_kernel<128, true>()) {
+            ds.status = NPA_ERR_UNSUPPORTED;  // a kernel's compiled shape does not match its launch plan
         } else {
             ds.status = NPA_OK;
         }
         ds.checked = true;
     }
     if (sm_count) *sm_count = ds.sm_count;
+    if (l2_bytes) *l2_bytes = ds.l2_bytes;
     return ds.status;
 }
 
@@ -236,8 +251,8 @@ npa_status validate_common(const void *q, const void *k, const void *v, void *o,
 npa_status launch(const void *q, const void *k, const void *v, const void *ks, const void *vs, void *o, int B,
                   int heads, int d, const Geo &g, int G, const npa_global_kv *gkv, int patch_begin, int patch_count,
                   npa_stream_t stream, float *md_part = nullptr) {
-    int sm_count = 0;
-    npa_status st = ensure_ready(&sm_count);
+    int sm_count = 0, l2_bytes = 0;
+    npa_status st = ensure_ready(&sm_count, &l2_bytes);
     if (st != NPA_OK) return st;
     const int nt = 2;  // query tiles per work unit
 
@@ -272,6 +287,12 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     prm.n_qblocks = (prm.tiles_c * prm.tiles_r + nt - 1) / nt;
     prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
     prm.wait_limit_ns = kWaitLimitNs;
+#ifdef NPA_DEBUG_BOUNDS
+    if (const unsigned stall_us = g_debug_stall_us.exchange(0)) {
+        prm.debug_stall = 1;
+        prm.wait_limit_ns = stall_us * 1000ull;
+    }
+#endif
 
     if ((long long)prm.nPh * prm.nPw > INT_MAX / 4) return NPA_ERR_UNSUPPORTED;
     prm.patch_begin = patch_begin;
@@ -285,8 +306,18 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     prm.n_units = (int)units;
     npa::order_patches(prm);
     // persistent grid: one CTA per multiprocessor (shared memory and TMEM
-    // admit one), each walking every gridDim.x-th unit
+    // admit one), each walking its host-built list of units (or every
+    // gridDim.x-th unit); when the keys and values of all heads do not fit in
+    // L2, the lists run head by head
     const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);
+#ifndef NPA_NO_SCHED_LISTS
+    if (!md_part) {
+#else
+    if (false) {
+#endif
+        const double kv_bytes = 4.0 * BH * (double)g.H * g.W * d + 4.0 * BH * (double)G * d;
+        npa::build_schedule(prm, (int)grid, kv_bytes > (double)l2_bytes);
+    }
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)BH};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)g.W * d * 2, (cuuint64_t)g.H * g.W * d * 2};
     const cuuint32_t qbox[4] = {64, (cuuint32_t)prm.qc, (cuuint32_t)prm.qr, 1};
@@ -736,6 +767,14 @@ npa_status npa_selftest_wait_timeout(uint32_t limit_us, npa_stream_t stream) {
     return e == cudaSuccess ? NPA_OK : NPA_ERR_CUDA;
 }
 
+#ifdef NPA_DEBUG_BOUNDS
+npa_status npa_debug_withhold_arrival_once(uint32_t wait_limit_us) {
+    if (wait_limit_us < 1 || wait_limit_us > 1000000) return NPA_ERR_INVALID_ARG;
+    g_debug_stall_us.store(wait_limit_us);
+    return NPA_OK;
+}
+#endif
+
 const char *npa_status_string(npa_status status) {
     switch (status) {
         case NPA_OK: return "NPA_OK";
@@ -744,6 +783,7 @@ const char *npa_status_string(npa_status status) {
         case NPA_ERR_MISALIGNED: return "NPA_ERR_MISALIGNED";
         case NPA_ERR_CUDA: return "NPA_ERR_CUDA";
         case NPA_ERR_DEVICE_TIMEOUT: return "NPA_ERR_DEVICE_TIMEOUT";
+        case NPA_ERR_DEVICE_BOUNDS: return "NPA_ERR_DEVICE_BOUNDS";
     }
     return "NPA_ERR_UNKNOWN";
 }

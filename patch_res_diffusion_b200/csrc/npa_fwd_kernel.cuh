@@ -64,61 +64,130 @@ __device__ unsigned int g_npa_status;  // first device-side error since last rea
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_npa_status, 0u, code); }
 
 constexpr unsigned int kErrDeviceTimeout = 5u;  // NPA_ERR_DEVICE_TIMEOUT
+constexpr unsigned int kErrDeviceBounds = 6u;   // NPA_ERR_DEVICE_BOUNDS (bounds-checking build)
+
+// Bounds-checking build (NPA_DEBUG_BOUNDS): every TMA box origin is checked
+// against its tensor's extent and every output row against the output's row
+// count. A failed check records NPA_ERR_DEVICE_BOUNDS; a load origin is then
+// clamped into the tensor (the copy still delivers its bytes, so no barrier
+// is left waiting) and a store is skipped. In the normal build these are
+// identities.
+__device__ __forceinline__ int bound_coord(int x, int extent) {
+#ifdef NPA_DEBUG_BOUNDS
+    if (x < 0 || x >= extent) {
+        record_error(kErrDeviceBounds);
+        return x < 0 ? 0 : extent - 1;
+    }
+#endif
+    return x;
+}
+
+__device__ __forceinline__ bool bound_row(bool valid, size_t row, size_t rows) {
+#ifdef NPA_DEBUG_BOUNDS
+    if (valid && row >= rows) {
+        record_error(kErrDeviceBounds);
+        return false;
+    }
+#endif
+    return valid;
+}
 
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
-// Kernel shape: D = head dimension, NT = query tiles per CTA (one softmax
-// warpgroup each), KB = keys per key block.
+// Kernel shape: D = head dimension, NT = query tiles per CTA, KB = keys per
+// key block. At d = 64 every query tile has two softmax warpgroups, one per
+// half of the block's score columns (kHalves = 2): the two warps of a
+// sub-partition that serve one tile evaluate their exponentials at the same
+// time, which keeps the exponential unit busier than one warp can, and they
+// agree on the block maximum (and at the end on the row sum) through a small
+// shared-memory exchange. At d = 128 one warpgroup serves a tile.
 template <int D, int NT, int KB>
 struct KCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(NT == 2 && KB == 128, "two query tiles per CTA, 128-key blocks");
+#ifndef NPA_D128_HALVES
+#define NPA_D128_HALVES 1
+#endif
+    static constexpr int kHalves = D == 64 ? 2 : NPA_D128_HALVES;  // softmax warpgroups per query tile
+    static_assert(kHalves == 1 || kHalves == 2, "column halves");
+    static constexpr int kCols = KB / kHalves;              // scores per thread per key block
+    static constexpr int kOCols = D / kHalves;              // output columns per thread
+    static constexpr int kSoftmaxWGs = NT * kHalves;
     static constexpr int kChunks = D / 64;                 // 64-element (128-byte) column blocks
     static constexpr int kQChunkBytes = 128 * 128;         // 128 query rows x 128 bytes
     static constexpr int kQTileBytes = kChunks * kQChunkBytes;
     static constexpr int kKVChunkBytes = KB * 128;         // KB key rows x 128 bytes
     static constexpr int kKVTileBytes = kChunks * kKVChunkBytes;
     static constexpr int kStages = D == 128 ? 2 : 4;
-    static constexpr int kThreads = 128 * (NT + 1);
-    static constexpr int kCtlWarp = 4 * NT;                // first warp of the control warpgroup
-    static constexpr uint32_t kRegsLaunch = 168;
-    static constexpr uint32_t kRegsSoftmax = 216;
-    static constexpr uint32_t kRegsCtl = 72;
-    static_assert(NT * 128 * kRegsSoftmax + 128 * kRegsCtl == kThreads * kRegsLaunch, "register split");
+    static constexpr int kThreads = 128 * (kSoftmaxWGs + 1);
+    static constexpr int kCtlWarp = 4 * kSoftmaxWGs;       // first warp of the control warpgroup
+    // registers per thread: at launch (the most __launch_bounds__ allows for
+    // kThreads; the host checks the compiled count before the first launch,
+    // since a split above the launch total would never complete), then after
+    // the control warpgroup gives registers back and the softmax warpgroups
+    // take them
+    static constexpr uint32_t kRegsLaunch = kHalves == 2 ? 96 : 168;
+    static constexpr uint32_t kRegsSoftmax = kHalves == 1 ? 216 : (D == 64 ? 104 : 96);
+    static constexpr uint32_t kRegsCtl = kHalves == 1 ? 72 : (D == 64 ? 64 : 96);
+    static_assert(kSoftmaxWGs * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
+    static_assert(kThreads * kRegsLaunch <= 65536, "register file");
+    // query buffers: at d = 64 two, so that the next unit's tiles load while
+    // the current unit runs (at d = 128 one: shared memory is full)
+#ifndef NPA_Q_BUFS
+#define NPA_Q_BUFS 2
+#endif
+    static constexpr int kQBufs = D == 64 ? NPA_Q_BUFS : 1;
+    static constexpr int kQBufBytes = NT * kQTileBytes;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = NT * kQTileBytes;
+    static constexpr int kOffK = kQBufs * kQBufBytes;
     static constexpr int kOffV = kOffK + kStages * kKVTileBytes;
     static constexpr int kOffBar = kOffV + kStages * kKVTileBytes;
     // barrier indices
-    static constexpr int bQFull = 0;
-    static constexpr int bQEmpty = 1;                  // Q buffer free (S issuer commit after a unit)
-    static constexpr int bKFull = 2;
+    static constexpr int bQFull = 0;                   // [kQBufs] query tiles landed
+    static constexpr int bQEmpty = bQFull + kQBufs;    // [kQBufs] buffer free (S issuer commit after a unit)
+    static constexpr int bKFull = bQEmpty + kQBufs;
     static constexpr int bKEmpty = bKFull + kStages;
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
     static constexpr int bSFull = bVEmpty + kStages;   // [NT] S_q written (MMA commit)
-    static constexpr int bSFree = bSFull + NT;         // [NT] S_q copied to registers (128 arrivals)
-    static constexpr int bPFull = bSFree + NT;         // [NT] P_q written (128 arrivals)
+    static constexpr int bSFree = bSFull + NT;         // [NT] S_q copied to registers (128 * kHalves arrivals)
+    static constexpr int bPFull = bSFree + NT;         // [NT] P_q written (128 * kHalves arrivals)
     static constexpr int bPFree = bPFull + NT;         // [NT] PV_q done (MMA commit)
-    // [NT][4] exponential-phase turn of warp k of warpgroup q (1 arrival): the
-    // turn passes between the warps that share a sub-partition's MUFU
+    // [NT][4] exponential-phase turn of warp k of tile q's warpgroups (one
+    // arrival per warpgroup of the tile): the turn passes between the warps
+    // that share a sub-partition's MUFU
     static constexpr int bTurn = bPFree + NT;
     static constexpr int bDrain = bTurn + 4 * NT;      // [2] one per MMA-issuing warp
-    static constexpr int kNumBars = bDrain + 2;
+    // [NT][4] (kHalves == 2) exchange between warp k of the two warpgroups of
+    // tile q (64 arrivals): block maxima, then the row sums
+    static constexpr int bXchg = bDrain + 2;
+    static constexpr int kNumBars = bXchg + 4 * NT;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+    static constexpr int kOffXchg = kOffMisc + 16;     // float [NT][kHalves][2 parities][128 rows]
+    static constexpr int kXchgBytes = kHalves == 2 ? NT * 2 * 2 * 128 * 4 : 0;
+    static constexpr int kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + slack for 1024-byte alignment
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     // tensor memory columns
     static constexpr uint32_t kTmemCols = 512;
     static constexpr bool kSeparateP = (D == 64);
-    // d = 64: the softmax warpgroups hand the exponential unit to each other
-    // in turn (measured +5..7% with two tiles); d = 128: the aliased-P issue
-    // order already alternates the tiles and the hand-off costs about 3%.
-    static constexpr bool kUseTurn = (D == 64);
+    // d = 64: the tiles' warpgroup pairs hand the exponential unit to each
+    // other in turn; d = 128: the aliased-P issue order already alternates the
+    // tiles and the hand-off costs about 3%.
+#ifndef NPA_D64_TURN
+#define NPA_D64_TURN 1
+#endif
+    static constexpr bool kUseTurn = (D == 64) && NPA_D64_TURN;
     __device__ static constexpr uint32_t col_s(int q) { return uint32_t(q * KB); }
     __device__ static constexpr uint32_t col_o(int q) { return uint32_t(NT * KB + q * D); }
     __device__ static constexpr uint32_t col_p(int q) {
         return kSeparateP ? uint32_t(NT * KB + NT * D + q * (KB / 2)) : col_s(q);
+    }
+    // P of column half h (keys [h * kCols, (h + 1) * kCols), packed bf16
+    // pairs: kCols / 2 columns): d = 64 in the separate P buffer, one after
+    // the other; d = 128 over the first columns of that half's own scores
+    // (which its warps have already read)
+    __device__ static constexpr uint32_t col_p_half(int q, int h) {
+        return kSeparateP ? col_p(q) + uint32_t(h * (kCols / 2)) : col_s(q) + uint32_t(h * kCols);
     }
     static_assert(!kSeparateP || NT * KB + NT * D + NT * (KB / 2) <= 512, "tensor memory columns");
     static_assert(kSeparateP || NT * KB + NT * D <= 512, "tensor memory columns");
@@ -126,8 +195,9 @@ struct KCfg {
 
 // ---------------------------------------------------------------------------
 // Persistent work loop. Every role of a CTA walks the same unit sequence
-// (blockIdx.x, blockIdx.x + gridDim.x, ...) and skips the same empty units, so
-// the roles agree on every barrier phase without exchanging unit indices.
+// (cta_unit: the host-built list of this CTA, or blockIdx.x, blockIdx.x +
+// gridDim.x, ...) and skips the same empty units, so the roles agree on every
+// barrier phase without exchanging unit indices.
 // Phases are counted across units: gb = key blocks processed so far by this
 // CTA (one S and one P per tile per block), uq = units processed so far.
 // ---------------------------------------------------------------------------
@@ -150,15 +220,16 @@ __device__ __forceinline__ void load_block(const FwdParams &p, const Work &w, in
     if (j < w.n_win) {
         const BlockGeom b = block_geom(p, w, j);
         const CUtensorMap *m = b.stale ? (is_v ? &p.tm_vs : &p.tm_ks) : (is_v ? &p.tm_v : &p.tm_k);
+        const int col = bound_coord(b.col, p.W), row = bound_coord(b.row, p.H), bh = bound_coord(w.bh, p.BH);
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_4d(dst + c * C::kKVChunkBytes, m, bar, c * 64, b.col, b.row, w.bh);
+            sm100::tma_load_4d(dst + c * C::kKVChunkBytes, m, bar, c * 64, col, row, bh);
     } else {
-        const int g0 = (j - w.n_win) * KB;
+        const int g0 = bound_coord((j - w.n_win) * KB, p.G), bh = bound_coord(w.bh, p.BH);
         const CUtensorMap *m = is_v ? &p.tm_gv : &p.tm_gk;
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c)
-            sm100::tma_load_3d(dst + c * C::kKVChunkBytes, m, bar, c * 64, g0, w.bh);
+            sm100::tma_load_3d(dst + c * C::kKVChunkBytes, m, bar, c * 64, g0, bh);
     }
 }
 
@@ -181,29 +252,39 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
     const uint32_t q_bytes = GQ ? uint32_t(C::kChunks * 128 * 128) : uint32_t(C::kChunks * p.qc * p.qr * 128);
     int nk = 0, nv = 0, uq = 0;  // K / V blocks and Q tile groups issued
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
         // the previous unit's last S products must be done with the Q buffer
-        if (uq > 0 && !sm100::mbar_wait(&bars[C::bQEmpty], (uq - 1) & 1, lim)) {
+        const int qbuf = uq % C::kQBufs, quse = uq / C::kQBufs;
+        uint8_t *qdst = smem + C::kOffQ + qbuf * C::kQBufBytes;
+        if (quse > 0 && !sm100::mbar_wait(&bars[C::bQEmpty + qbuf], (quse - 1) & 1, lim)) {
             ok = false;
             break;
         }
-        sm100::mbar_arrive_expect_tx(&bars[C::bQFull], NT * q_bytes);
+        sm100::mbar_arrive_expect_tx(&bars[C::bQFull + qbuf], NT * q_bytes);
+        // a unit's query tile past the patch's last (its outputs are not
+        // stored) loads the unit's first tile again, so every box starts
+        // inside the tensor
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
+            const int bh = bound_coord(w.bh, p.BH);
             if (GQ) {
+                const int tq = w.tile0 + t < p.gq_tiles ? w.tile0 + t : w.tile0;
+                const int g0 = bound_coord(tq * 128, p.G);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_3d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_gq,
-                                       &bars[C::bQFull], c * 64, (w.tile0 + t) * 128, w.bh);
+                    sm100::tma_load_3d(qdst + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_gq,
+                                       &bars[C::bQFull + qbuf], c * 64, g0, bh);
             } else {
                 int row0, col0;
-                q_tile_origin(p, w, w.tile0 + t, &row0, &col0);
+                q_tile_origin(p, w, q_tile_valid(p, w, w.tile0 + t) ? w.tile0 + t : w.tile0, &row0, &col0);
+                row0 = bound_coord(row0, p.H);
+                col0 = bound_coord(col0, p.W);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_4d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_q,
-                                       &bars[C::bQFull], c * 64, col0, row0, w.bh);
+                    sm100::tma_load_4d(qdst + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_q,
+                                       &bars[C::bQFull + qbuf], c * 64, col0, row0, bh);
             }
         }
         ++uq;
@@ -235,7 +316,10 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
     }
     // Drain: every issued copy must have landed before the CTA may exit
     // (immediate on the normal path, where the consumers already saw them).
-    if (uq > 0) sm100::mbar_wait(&bars[C::bQFull], (uq - 1) & 1, lim);
+    for (int b = 0; b < C::kQBufs && b < uq; ++b) {  // the last unit that used buffer b
+        const int u_last = uq - 1 - ((uq - 1 - b) % C::kQBufs);
+        sm100::mbar_wait(&bars[C::bQFull + b], (u_last / C::kQBufs) & 1, lim);
+    }
     for (int s = 0; s < C::kStages; ++s) {
         if (nk > s) sm100::mbar_wait(&bars[C::bKFull + s], ((nk - 1 - s) / C::kStages) & 1, lim);
         if (nv > s) sm100::mbar_wait(&bars[C::bVFull + s], ((nv - 1 - s) / C::kStages) & 1, lim);
@@ -265,15 +349,17 @@ template <int D, int NT, int KB>
 __device__ __forceinline__ void issue_pv(uint32_t tmem, int q, uint64_t vdesc, bool accumulate) {
     using C = KCfg<D, NT, KB>;
     constexpr uint32_t kIdO = sm100::idesc_bf16_f32(128, D, false, true);  // O += P V, V MN-major
+    constexpr int kStepsPerHalf = C::kCols / 16;  // K16 steps per column half of P
 #pragma unroll
     for (int kk = 0; kk < KB / 16; ++kk)
-        sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p(q) + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), kIdO,
-                      (accumulate || kk > 0) ? 1u : 0u);
+        sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p_half(q, kk / kStepsPerHalf) + (kk % kStepsPerHalf) * 8,
+                      vdesc + uint64_t((kk * 2048) >> 4), kIdO, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 struct OperandDescs {
     uint64_t q0, k0, v0;  // Q tile 0, K and V stage 0
     uint64_t qtile;       // descriptor increment from one Q tile to the next
+    uint64_t qbuf;        // descriptor increment from one Q buffer to the next
     uint64_t stage;       // descriptor increment from one K/V stage to the next
 };
 
@@ -287,6 +373,7 @@ __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
     d.k0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffK), 16, 1024);
     d.v0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffV), C::kKVChunkBytes, 1024);
     d.qtile = uint64_t(C::kQTileBytes >> 4);
+    d.qbuf = uint64_t(C::kQBufBytes >> 4);
     d.stage = uint64_t(C::kKVTileBytes >> 4);
     return d;
 }
@@ -304,11 +391,13 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
     const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0, uq = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
-        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
+        const int qbuf = uq % C::kQBufs;
+        ok = sm100::mbar_wait(&bars[C::bQFull + qbuf], (uq / C::kQBufs) & 1, lim);
         ++uq;
+        const uint64_t qd = dd.q0 + qbuf * dd.qbuf;
         for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
             if (*abort_flag) {
                 ok = false;
@@ -320,12 +409,12 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
                 if (gb > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (gb - 1) & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + s * dd.stage);
+                issue_s<D, NT, KB>(tmem, q, qd + q * dd.qtile, dd.k0 + s * dd.stage);
                 sm100::tc_commit(&bars[C::bSFull + q]);
             }
             if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
         }
-        if (ok) sm100::tc_commit(&bars[C::bQEmpty]);  // this unit's Q is no longer read
+        if (ok) sm100::tc_commit(&bars[C::bQEmpty + qbuf]);  // this unit's Q is no longer read
     }
     if (!ok) {
         record_error(kErrDeviceTimeout);
@@ -344,7 +433,7 @@ __device__ void run_mma_pv(const FwdParams &p, uint8_t *smem, uint64_t *bars, ui
     const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
         for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
@@ -382,12 +471,14 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
     const OperandDescs dd = make_descs<D, NT, KB>(smem);
     int gb = 0, uq = 0;  // gb: global index of block j = 0 of the current unit
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
         const int n = w.je - w.jb;  // blocks of this unit, counted from its first
-        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
+        const int qbuf = uq % C::kQBufs;
+        ok = sm100::mbar_wait(&bars[C::bQFull + qbuf], (uq / C::kQBufs) & 1, lim);
         ++uq;
+        const uint64_t qd = dd.q0 + qbuf * dd.qbuf;
         sm100::tc_fence_after();
         for (int j = 0; ok && j <= n; ++j) {
             if (*abort_flag) {
@@ -413,13 +504,13 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
                     sm100::tc_commit(&bars[C::bPFree + q]);
                 }
                 if (j < n) {
-                    issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + (g % C::kStages) * dd.stage);
+                    issue_s<D, NT, KB>(tmem, q, qd + q * dd.qtile, dd.k0 + (g % C::kStages) * dd.stage);
                     sm100::tc_commit(&bars[C::bSFull + q]);
                 }
             }
             if (!ok) break;
             if (j < n) sm100::tc_commit(&bars[C::bKEmpty + g % C::kStages]);
-            if (j == n - 1) sm100::tc_commit(&bars[C::bQEmpty]);
+            if (j == n - 1) sm100::tc_commit(&bars[C::bQEmpty + qbuf]);
             if (j > 0) sm100::tc_commit(&bars[C::bVEmpty + (g - 1) % C::kStages]);
         }
         gb += n;
@@ -456,8 +547,47 @@ __device__ __forceinline__ float row_max(const float (&s)[KB]) {
     return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
 }
 
-// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum returned.
-template <int KB>
+// Exponentials on the FMA pipe, to offload the special-function unit (MUFU),
+// which bounds the d = 64 softmax: every kPolyEvery-th pair of a thread's
+// exponentials in blocks without masked keys (0: none). Build option
+// NPA_EXP_POLY_EVERY.
+#ifndef NPA_EXP_POLY_EVERY
+#define NPA_EXP_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = NPA_EXP_POLY_EVERY;
+
+// Minimax coefficients (relative error on [-1/2, 1/2], found by the Remez
+// exchange; largest relative error 7.5e-5) of the cubic c0 + c1 f + c2 f^2 +
+// c3 f^3 that approximates 2^f.
+constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
+
+// 2^x for a pair of finite arguments on the FMA pipe. x is clamped below at
+// -125 (the result is then about 2^-125, negligible next to the row sum,
+// which is at least 1), split as x = j + f with j = rint(x) - the float32
+// addition of 1.5 * 2^23 rounds to an integer held in the low mantissa bits -
+// and f = x - j in [-1/2, 1/2]; 2^f comes from the cubic above and 2^j is
+// added to its exponent field (j << 23; the constant's own bits shift out).
+__device__ __forceinline__ void exp2_fma_x2(uint64_t x2, float &p0, float &p1) {
+    float x0, x1;
+    sm100::unpack_f32x2(x2, x0, x1);
+    const uint64_t xc = sm100::pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = sm100::add_f32x2(xc, sm100::pack_f32x2(12582912.f, 12582912.f));
+    const uint64_t j = sm100::add_f32x2(t, sm100::pack_f32x2(-12582912.f, -12582912.f));
+    const uint64_t f = sm100::fma_f32x2(j, sm100::pack_f32x2(-1.f, -1.f), xc);
+    uint64_t q = sm100::fma_f32x2(sm100::pack_f32x2(kExp2C3, kExp2C3), f, sm100::pack_f32x2(kExp2C2, kExp2C2));
+    q = sm100::fma_f32x2(q, f, sm100::pack_f32x2(kExp2C1, kExp2C1));
+    q = sm100::fma_f32x2(q, f, sm100::pack_f32x2(kExp2C0, kExp2C0));
+    float q0, q1, t0, t1;
+    sm100::unpack_f32x2(q, q0, q1);
+    sm100::unpack_f32x2(t, t0, t1);
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum
+// returned. POLY > 0: every POLY-th pair on the FMA pipe (no -inf scores).
+template <int KB, int POLY>
 __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2]) {
     const float neg = (ref == -INFINITY) ? 0.f : -ref;
     const uint64_t c2 = sm100::pack_f32x2(c, c);
@@ -466,10 +596,15 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
 #pragma unroll
     for (int i = 0; i < KB / 2; ++i) {
         const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
-        float x0, x1;
-        sm100::unpack_f32x2(x2, x0, x1);
-        const float p0 = sm100::ex2_approx(x0);
-        const float p1 = sm100::ex2_approx(x1);
+        float p0, p1;
+        if (POLY > 0 && i % (POLY > 0 ? POLY : 1) == POLY - 1) {
+            exp2_fma_x2(x2, p0, p1);
+        } else {
+            float x0, x1;
+            sm100::unpack_f32x2(x2, x0, x1);
+            p0 = sm100::ex2_approx(x0);
+            p1 = sm100::ex2_approx(x1);
+        }
         pk[i] = sm100::pack_bf16x2(p0, p1);
         acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
     }
@@ -481,23 +616,47 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
     return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
+// Exchange between the two warps (one per column half) that serve the same
+// 32 rows of a query tile: each writes its value for its row, arrives on the
+// pair's barrier (release) and, once the phase completes (acquire), reads the
+// partner's. Slots alternate by phase parity, so a partner one phase ahead
+// cannot overwrite a value before it is read. False if the wait ran out.
+__device__ __forceinline__ bool pair_exchange(float *xbuf, uint64_t *bar, int h, int row, int xp, float mine,
+                                              float &other, uint64_t lim) {
+    const int par = xp & 1;
+    xbuf[(h * 2 + par) * 128 + row] = mine;
+    sm100::mbar_arrive(bar);
+    if (!warp_wait(bar, par, lim)) return false;
+    other = xbuf[((1 - h) * 2 + par) * 128 + row];
+    return true;
+}
+
+// Softmax and epilogue of softmax warpgroup g: query tile q = g / kHalves,
+// score columns [h * kCols, (h + 1) * kCols) of every key block and output
+// columns [h * kOCols, (h + 1) * kOCols), h = g % kHalves. Each thread owns one
+// query row (its TMEM lane).
 template <int D, int NT, int KB, bool GQ, bool MD>
-__device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
-                            int q) {
+__device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
+                            volatile uint32_t *abort_flag, int g) {
     using C = KCfg<D, NT, KB>;
+    constexpr int kC = C::kCols;
+    const int q = g / C::kHalves, h = g % C::kHalves;
     const uint64_t lim = p.wait_limit_ns;
     const int row = threadIdx.x & 127;
     const bool lane0 = (threadIdx.x & 31) == 0;
     const int warp_in_group = (threadIdx.x >> 5) & 3;
     const uint32_t lane_off = uint32_t(warp_in_group) * 32u << 16;
-    const uint32_t tS = tmem + lane_off + C::col_s(q);
-    const uint32_t tO = tmem + lane_off + C::col_o(q);
-    const uint32_t tP = tmem + lane_off + C::col_p(q);
+    const uint32_t tS = tmem + lane_off + C::col_s(q) + uint32_t(h * kC);
+    const uint32_t tO = tmem + lane_off + C::col_o(q) + uint32_t(h * C::kOCols);
+    const uint32_t tP = tmem + lane_off + C::col_p_half(q, h);
+    float *xbuf = reinterpret_cast<float *>(smem + C::kOffXchg) + q * (2 * 2 * 128);
+    uint64_t *xbar = &bars[C::bXchg + 4 * q + warp_in_group];
     const float sl2 = p.scale_log2;
     const int kc = 1 << p.kc_log2;
     int gb = 0;  // global index (across units) of the current block
+    int xp = 0;  // exchange phases completed by this warp pair
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < p.n_units; unit += gridDim.x) {
+    for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
     const Work w = decode<GQ>(p, unit);
     if (!unit_has_work<NT, GQ>(p, w)) continue;
     // window block coordinates, advanced without divisions: column block,
@@ -510,19 +669,22 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
     }
     float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
     float R_prev = -INFINITY;  // reference that O and l are currently expressed in
-    float l = 0.f;
+    float l = 0.f;             // this column half's share of the row sum
     for (int j = w.jb; j < w.je; ++j, ++gb) {
         if (!warp_wait(&bars[C::bSFull + q], gb & 1, lim)) {
             ok = false;
             break;
         }
         sm100::tc_fence_after();
-        float s[KB];
+        float s[kC];
         {
-            uint32_t sr[KB];
-            sm100::tmem_ld128(tS, sr);
+            uint32_t sr[kC];
+            if constexpr (kC == 128)
+                sm100::tmem_ld128(tS, sr);
+            else
+                sm100::tmem_ld64(tS, sr);
 #pragma unroll
-            for (int i = 0; i < KB; ++i) s[i] = __uint_as_float(sr[i]);
+            for (int i = 0; i < kC; ++i) s[i] = __uint_as_float(sr[i]);
         }
         if (C::kSeparateP) {
             // S_q may be overwritten by the next block's scores
@@ -530,14 +692,19 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             sm100::mbar_arrive(&bars[C::bSFree + q]);
         }
         // keys of this block outside its row segment or the window (or past
-        // the last global token) get -inf
+        // the last global token) get -inf; this half's key i is block key
+        // h * kC + i
+        bool masked = false;  // some key of this block (either half) is outside its set
         if (j < w.n_win) {
             const int vc = w.wc1 - (w.wc0 + (btc << p.kc_log2));
             const int vr = bend - brow;
-            if (vc < kc || vr < p.kr) {
+            masked = vc < kc || vr < p.kr;
+            if (masked) {
 #pragma unroll
-                for (int i = 0; i < KB; ++i)
-                    if ((i & (kc - 1)) >= vc || (i >> p.kc_log2) >= vr) s[i] = -INFINITY;
+                for (int i = 0; i < kC; ++i) {
+                    const int key = h * kC + i;
+                    if ((key & (kc - 1)) >= vc || (key >> p.kc_log2) >= vr) s[i] = -INFINITY;
+                }
             }
             if (++btc == w.wtc) {
                 btc = 0;
@@ -548,29 +715,44 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
                 }
             }
         } else {
-            const int vg = p.G - (j - w.n_win) * KB;
-            if (vg < KB) {
+            const int vg = p.G - (j - w.n_win) * KB - h * kC;
+            masked = p.G - (j - w.n_win) * KB < KB;
+            if (vg < kC) {
 #pragma unroll
-                for (int i = 0; i < KB; ++i)
+                for (int i = 0; i < kC; ++i)
                     if (i >= vg) s[i] = -INFINITY;
             }
         }
-        // block maximum and the reference for this block's P (lazy: the
-        // reference moves only when the maximum grows by more than kRescaleLog2)
-        const float bm = row_max<KB>(s) * sl2;
+        // block maximum over both column halves, and the reference for this
+        // block's P (lazy: the reference moves only when the maximum grows by
+        // more than kRescaleLog2); both halves take the same decision
+        float bmax = row_max<kC>(s);
+        if constexpr (C::kHalves == 2) {
+            float other;
+            if (!pair_exchange(xbuf, xbar, h, row, xp, bmax, other, lim)) {
+                ok = false;
+                break;
+            }
+            ++xp;
+            bmax = fmaxf(bmax, other);
+        }
+        const float bm = bmax * sl2;
         if (bm > R + kRescaleLog2) R = bm;
-        // wait for this warpgroup's turn on the exponential unit (the turn
-        // goes round the warpgroups in order, block by block)
+        // wait for this tile's turn on the exponential unit (the turn goes
+        // round the tiles in order, block by block)
         if (C::kUseTurn && (q > 0 || gb > 0) &&
             !warp_wait(&bars[C::bTurn + 4 * q + warp_in_group], (q == 0 ? gb - 1 : gb) & 1, lim)) {
             ok = false;
             break;
         }
-        uint32_t pk[KB / 2];
-        const float blk_sum = exp_block<KB>(s, sl2, R, pk);
-        // pass the turn to the next warpgroup's warp on this sub-partition
-        // once the whole block is issued (handing it over at 3/4 or 7/8 of
-        // the block measured 16-17% slower)
+        uint32_t pk[kC / 2];
+        float blk_sum;
+        if (kPolyEvery > 0 && C::kSeparateP && !masked)
+            blk_sum = exp_block<kC, (C::kSeparateP ? kPolyEvery : 0)>(s, sl2, R, pk);
+        else
+            blk_sum = exp_block<kC, 0>(s, sl2, R, pk);
+        // pass the turn to the next tile's warps on this sub-partition once
+        // the whole block is issued
         if (C::kUseTurn) {
             __syncwarp();
             if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
@@ -586,7 +768,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         }
         if (j > w.jb && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < C::kOCols / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
 #pragma unroll
@@ -595,30 +777,52 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
         }
         l = l * alpha + blk_sum;
-        sm100::tmem_st64(tP, pk);
+        if constexpr (kC == 128)
+            sm100::tmem_st64(tP, pk);
+        else
+            sm100::tmem_st32(tP, pk);
         sm100::tc_fence_before();
-        sm100::mbar_arrive(&bars[C::bPFull + q]);
+#ifdef NPA_DEBUG_BOUNDS
+        // abort-path test: the last tile of CTA 0 never announces its second
+        // block's P, so the P.V issuer's bounded wait runs out and every role
+        // drains and stops (no copy or product is left in flight)
+        if (!(p.debug_stall && blockIdx.x == 0 && q == NT - 1 && gb == 1))
+#endif
+            sm100::mbar_arrive(&bars[C::bPFull + q]);
         R_prev = R;
     }
     // the last PV of this tile completes phase gb-1 of P_free
     if (ok && !warp_wait(&bars[C::bPFree + q], (gb - 1) & 1, lim)) ok = false;
     if (!ok) break;
     sm100::tc_fence_after();
-    // epilogue: O / l -> bf16 -> the query's token position
+    // the row sum over both column halves, added in the same order by both
+    if constexpr (C::kHalves == 2) {
+        float other;
+        if (!pair_exchange(xbuf, xbar, h, row, xp, l, other, lim)) {
+            ok = false;
+            break;
+        }
+        ++xp;
+        l = h == 0 ? l + other : other + l;
+    }
+    // epilogue: O / l -> bf16 -> the query's token position (this half's
+    // output columns)
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const int t = w.tile0 + q;
+    const int c0 = h * C::kOCols;
     bool valid;
     size_t out_row;
     if (GQ) {
-        const int g = t * 128 + row;
-        valid = t < p.gq_tiles && g < p.G;
-        out_row = (size_t)w.bh * p.G + g;
+        const int gr = t * 128 + row;
+        valid = t < p.gq_tiles && gr < p.G;
+        out_row = (size_t)w.bh * p.G + gr;
         if (p.n_splits > 1) {
             // a key-range split: unnormalised O with its reference maximum and row sum
             const size_t prow = (size_t)w.split * p.BH * p.G + out_row;
-            float4 *part = reinterpret_cast<float4 *>(p.o_part + prow * D);
+            valid = bound_row(valid, prow, (size_t)p.n_splits * p.BH * p.G);
+            float4 *part = reinterpret_cast<float4 *>(p.o_part + prow * D + c0);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < C::kOCols / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
                 if (valid) {
@@ -628,7 +832,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
                                                       __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
                 }
             }
-            if (valid) *reinterpret_cast<float2 *>(p.ml + prow * 2) = make_float2(R_prev, l);
+            if (valid && h == 0) *reinterpret_cast<float2 *>(p.ml + prow * 2) = make_float2(R_prev, l);
             continue;
         }
     } else {
@@ -646,9 +850,10 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             const int rh = md_axis_offset(p.H, p.Ph, p.mh, patch / p.nPw);
             const int cw = md_axis_offset(p.W, p.Pw, p.mw, patch % p.nPw);
             const size_t prow = ((size_t)w.bh * p.md_rows + (rh + grow - w.wr0)) * p.md_tw + (cw + gcol - w.wc0);
-            float4 *part = reinterpret_cast<float4 *>(p.md_part + prow * D);
+            valid = bound_row(valid, prow, (size_t)p.BH * p.md_rows * p.md_tw);
+            float4 *part = reinterpret_cast<float4 *>(p.md_part + prow * D + c0);
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < C::kOCols / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
                 if (valid) {
@@ -662,9 +867,10 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             continue;
         }
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D);
+    valid = bound_row(valid, out_row, GQ ? (size_t)p.BH * p.G : (size_t)p.BH * p.H * p.W);
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D + c0);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < C::kOCols / 32; ++c) {
         uint32_t o[32];
         sm100::tmem_ld32(tO + c * 32, o);
         if (valid) {
@@ -703,8 +909,10 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        sm100::mbar_init(&bars[C::bQFull], 1);
-        sm100::mbar_init(&bars[C::bQEmpty], 1);
+        for (int b = 0; b < C::kQBufs; ++b) {
+            sm100::mbar_init(&bars[C::bQFull + b], 1);
+            sm100::mbar_init(&bars[C::bQEmpty + b], 1);
+        }
         for (int s = 0; s < C::kStages; ++s) {
             sm100::mbar_init(&bars[C::bKFull + s], 1);
             sm100::mbar_init(&bars[C::bKEmpty + s], 1);
@@ -713,10 +921,13 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
         }
         for (int q = 0; q < NT; ++q) {
             sm100::mbar_init(&bars[C::bSFull + q], 1);
-            sm100::mbar_init(&bars[C::bSFree + q], 128);
-            sm100::mbar_init(&bars[C::bPFull + q], 128);
+            sm100::mbar_init(&bars[C::bSFree + q], 128 * C::kHalves);
+            sm100::mbar_init(&bars[C::bPFull + q], 128 * C::kHalves);
             sm100::mbar_init(&bars[C::bPFree + q], 1);
-            for (int k = 0; k < 4; ++k) sm100::mbar_init(&bars[C::bTurn + 4 * q + k], 1);
+            for (int k = 0; k < 4; ++k) {
+                sm100::mbar_init(&bars[C::bTurn + 4 * q + k], C::kHalves);
+                sm100::mbar_init(&bars[C::bXchg + 4 * q + k], 64);  // used when kHalves == 2
+            }
         }
         sm100::mbar_init(&bars[C::bDrain], 1);
         sm100::mbar_init(&bars[C::bDrain + 1], 1);
@@ -747,7 +958,7 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
         }
     } else {
         sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D, NT, KB, GQ, MD>(p, bars, tmem, abort_flag, warp >> 2);
+        run_softmax<D, NT, KB, GQ, MD>(p, smem, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();

@@ -28,6 +28,14 @@ namespace npa {
 // natural order.
 constexpr int kMaxPatchOrder = 256;
 constexpr int kMaxCostClasses = 16;
+// A host-built per-CTA unit list covers launches of up to this many units and
+// CTAs (it travels in the kernel parameters); larger launches run the units
+// round robin.
+constexpr int kMaxSchedUnits = 7168;
+constexpr int kMaxSchedCtas = 160;
+// Scheduling cost of a unit beyond its key blocks (query load, pipeline
+// refill, epilogue), in key blocks.
+constexpr int kUnitOverheadBlocks = 2;
 
 struct FwdParams {
     CUtensorMap tm_q;   // 4D {d, W, H, B*heads}, box {64, qc, qr, 1}, 128B swizzle
@@ -69,6 +77,13 @@ struct FwdParams {
     int md;
     int md_rows, md_tw;              // sum of window heights / widths over the patch rows / columns
     float *md_part;                  // [B*heads][md_rows][md_tw][d]
+    // Per-CTA unit lists (n_sched > 0): CTA c runs units sched[cta_first[c]],
+    // ..., sched[cta_first[c + 1] - 1] in that order. n_sched == 0: CTA c
+    // runs units c, c + gridDim.x, c + 2 gridDim.x, ...
+    int debug_stall;  // bounds-checking build: CTA 0 withholds one P_full arrival (abort-path test)
+    int n_sched;
+    unsigned short cta_first[kMaxSchedCtas + 1];
+    unsigned short sched[kMaxSchedUnits];
 };
 
 // The window's rows are walked as three segments: [seg[0], seg[1]) and
@@ -197,6 +212,84 @@ __host__ __device__ inline int unit_patch(const FwdParams &p, int unit, int *bh)
         rank = rest / p.BH;
     }
     return p.n_perm ? int(p.patch_order[rank]) : p.patch_begin + rank;
+}
+
+// Host: the per-CTA unit lists. Units are taken in one global order and each
+// goes to the CTA that becomes free first (list scheduling on the predicted
+// cost: the key blocks of the unit's window plus kUnitOverheadBlocks), so the
+// CTAs finish together and, at any moment, the running units lie close
+// together in the global order. The global order is the unit numbering
+// (cost class, then batch*head, then patch, then query-tile group: cheapest
+// last) or, with head_major, batch*head first and then cost class, patch and
+// query-tile group, so that the units running at one time share one or two
+// heads' keys and values (a whole head's windows stay in L2, instead of being
+// read again for every cost class). Needs order_patches() done with a class
+// table; leaves n_sched = 0 (round robin) otherwise or past the table sizes.
+inline void build_schedule(FwdParams &p, int grid, bool head_major) {
+    p.n_sched = 0;
+    if (p.n_cls == 0 || p.n_units > kMaxSchedUnits || grid > kMaxSchedCtas || grid < 1) return;
+    static thread_local unsigned short order[kMaxSchedUnits];
+    static thread_local unsigned short owner[kMaxSchedUnits];
+    int n = 0;
+    const int nq = p.n_qblocks;
+    if (head_major) {
+        for (int bh = 0; bh < p.BH; ++bh)
+            for (int c = 0; c < p.n_cls; ++c) {
+                const int cnt = p.cls_rank0[c + 1] - p.cls_rank0[c];
+                for (int k = 0; k < cnt; ++k)
+                    for (int qb = 0; qb < nq; ++qb)
+                        order[n++] = (unsigned short)((p.BH * p.cls_rank0[c] + bh * cnt + k) * nq + qb);
+            }
+    } else {
+        for (int u = 0; u < p.n_units; ++u) order[n++] = (unsigned short)u;
+    }
+    // binary min-heap of (finish time, cta), ties to the lower CTA index
+    long long tfin[kMaxSchedCtas];
+    int heap[kMaxSchedCtas], count[kMaxSchedCtas];
+    for (int c = 0; c < grid; ++c) {
+        tfin[c] = 0;
+        heap[c] = c;
+        count[c] = 0;
+    }
+    auto less = [&](int a, int b) { return tfin[a] < tfin[b] || (tfin[a] == tfin[b] && a < b); };
+    for (int i = 0; i < n; ++i) {
+        int bh;
+        const int c = heap[0];
+        owner[i] = (unsigned short)c;
+        ++count[c];
+        tfin[c] += patch_cost(p, unit_patch(p, order[i], &bh)) + kUnitOverheadBlocks;
+        for (int k = 0;;) {  // sift the root down
+            const int l = 2 * k + 1, r = l + 1;
+            int m = k;
+            if (l < grid && less(heap[l], heap[m])) m = l;
+            if (r < grid && less(heap[r], heap[m])) m = r;
+            if (m == k) break;
+            const int t = heap[k];
+            heap[k] = heap[m];
+            heap[m] = t;
+            k = m;
+        }
+    }
+    p.cta_first[0] = 0;
+    for (int c = 0; c < grid; ++c) p.cta_first[c + 1] = (unsigned short)(p.cta_first[c] + count[c]);
+    int fill[kMaxSchedCtas];
+    for (int c = 0; c < grid; ++c) fill[c] = p.cta_first[c];
+    for (int i = 0; i < n; ++i) p.sched[fill[owner[i]]++] = order[i];
+    p.n_sched = n;
+}
+
+// The i-th unit of this CTA's work, or -1 past its last.
+__device__ __forceinline__ int cta_unit(const FwdParams &p, int i) {
+#ifdef __CUDA_ARCH__
+    if (p.n_sched) {
+        const int k = p.cta_first[blockIdx.x] + i;
+        return k < p.cta_first[blockIdx.x + 1] ? int(p.sched[k]) : -1;
+    }
+    const int u = blockIdx.x + i * gridDim.x;
+    return u < p.n_units ? u : -1;
+#else
+    return -1;
+#endif
 }
 
 __host__ __device__ inline Work decode_work(const FwdParams &p, int unit) {

@@ -32,21 +32,33 @@ def L():
 
 
 def test_header_declares_the_bound_symbols():
-    assert header_functions() == sorted(npa.EXPORTED_SYMBOLS)
+    assert header_functions() == sorted(npa.EXPORTED_SYMBOLS + npa.DEBUG_ONLY_SYMBOLS)
+
+
+def _exported(path):
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True, check=True).stdout
+    return {line.split()[-1] for line in out.splitlines() if " T " in line}
 
 
 def test_library_exports_every_header_symbol(L):
-    out = subprocess.run(["nm", "-D", "--defined-only", npa.LIB_PATH], capture_output=True, text=True,
-                         check=True).stdout
-    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
-    for name in header_functions():
+    exported = _exported(npa.LIB_PATH)
+    for name in npa.EXPORTED_SYMBOLS:
         assert name in exported, name
         assert getattr(L, name) is not None
+    for name in npa.DEBUG_ONLY_SYMBOLS:   # the bounds-checking build's own entry points
+        assert name not in exported, name
+
+
+def test_bounds_checking_library_exports_every_header_symbol(L):
+    exported = _exported(npa.DEBUG_LIB_PATH)
+    for name in header_functions():
+        assert name in exported, name
 
 
 def test_status_strings(L):
     for code, name in [(0, "NPA_OK"), (1, "NPA_ERR_INVALID_ARG"), (2, "NPA_ERR_UNSUPPORTED"),
-                       (3, "NPA_ERR_MISALIGNED"), (4, "NPA_ERR_CUDA"), (5, "NPA_ERR_DEVICE_TIMEOUT")]:
+                       (3, "NPA_ERR_MISALIGNED"), (4, "NPA_ERR_CUDA"), (5, "NPA_ERR_DEVICE_TIMEOUT"),
+                       (6, "NPA_ERR_DEVICE_BOUNDS")]:
         assert npa.npa_status_string(code) == name
     assert npa.npa_status_string(99) == "NPA_ERR_UNKNOWN"
 

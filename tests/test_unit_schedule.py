@@ -1,7 +1,9 @@
 """The persistent kernel's work-unit order (host arithmetic, no GPU): every
 (batch*head, patch, query-tile pair) of the computed patch range is decoded
 exactly once, cheapest units last, for NPA and PCPP geometries with ragged
-patches, patch ranges and more cost classes than the class table holds."""
+patches, patch ranges and more cost classes than the class table holds; the
+host-built per-CTA unit lists hold every unit once, balance the predicted
+cost, and (head by head) keep the running units on one or two heads."""
 import os
 import shutil
 import subprocess
@@ -26,7 +28,8 @@ def run(exe, *args):
     out = subprocess.run([exe, *map(str, args)], capture_output=True, text=True)
     assert out.returncode == 0, out.stdout + out.stderr
     f = out.stdout.split()
-    return {"units": int(f[2]), "ordered": int(f[4]), "classes": int(f[6]), "wave_heads": int(f[8])}
+    return {"units": int(f[2]), "ordered": int(f[4]), "classes": int(f[6]), "wave_heads": int(f[8]),
+            "sched": int(f[10]), "balance": float(f[12]), "first_heads": int(f[14]), "bound": float(f[16])}
 
 
 # BH, H, W, Ph, Pw, mh, mw, kb, kc_log2, tiles_per_unit, n_qblocks, patch_begin, patch_count
@@ -81,3 +84,28 @@ def test_overlapping_window_cover_range(checker, L, P, m):
     overlapping-window combine) equals a scan over every window."""
     out = subprocess.run([checker, "cover", str(L), str(P), str(m)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.startswith("ok"), out.stdout + out.stderr
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+@pytest.mark.parametrize("head_major", [0, 1])
+def test_per_cta_lists_hold_every_unit_once(checker, name, head_major):
+    r = run(checker, *CASES[name], 148, head_major)
+    if r["classes"] == 0 or r["units"] > 7168:
+        assert r["sched"] == 0          # no class table or too many units: round robin
+    else:
+        assert r["sched"] == r["units"]
+        # list scheduling: no CTA's predicted finish is more than one unit's
+        # cost above the mean
+        assert r["balance"] <= r["bound"] + 1e-9
+
+
+def test_head_major_lists_keep_running_units_on_few_heads(checker):
+    """SDXL 4096^2: 256 units per head over 148 CTAs; head by head, the first
+    units of all CTAs lie in at most two heads, and the predicted balance is
+    within 1.5% of perfect (round robin in the class order: 1.2%)."""
+    r = run(checker, *CASES["npa_sdxl_4096"], 148, 1)
+    assert r["sched"] == 5120
+    assert r["first_heads"] <= 2
+    assert r["balance"] < 1.015
+    r = run(checker, *CASES["pcpp_4x32"], 148, 0)
+    assert r["balance"] < 1.035

@@ -44,8 +44,10 @@ static int check_cover(int L, int P, int m) {
 int main(int argc, char **argv) {
     if (argc == 5 && std::strcmp(argv[1], "cover") == 0)
         return check_cover(std::atoi(argv[2]), std::atoi(argv[3]), std::atoi(argv[4]));
-    if (argc != 15) {
-        std::fprintf(stderr, "usage: BH H W Ph Pw mh mw kb kc_log2 tiles_per_unit n_qblocks patch_begin patch_count wave\n");
+    if (argc != 15 && argc != 16) {
+        std::fprintf(stderr,
+                     "usage: BH H W Ph Pw mh mw kb kc_log2 tiles_per_unit n_qblocks patch_begin patch_count wave "
+                     "[head_major]\n");
         return 2;
     }
     int a[14];
@@ -96,7 +98,42 @@ int main(int argc, char **argv) {
         }
         if (u < wave) wave_bh.insert(w.bh);
     }
-    std::printf("ok units %d ordered %d classes %d wave_heads %d\n", p.n_units, p.n_perm, p.n_cls,
-                (int)wave_bh.size());
+    // the per-CTA lists (wave = CTA count): every unit exactly once; the
+    // predicted finish time of the busiest CTA over the mean (and its list
+    // scheduling bound: the mean plus the costliest unit); the heads the first
+    // unit of every CTA touches
+    const int grid = p.n_units < wave ? p.n_units : wave;
+    npa::build_schedule(p, grid, argc == 16 && std::atoi(argv[15]) != 0);
+    double balance = 0.0, bound = 0.0;
+    std::set<int> first_bh;
+    if (p.n_sched) {
+        if (p.n_sched != p.n_units || p.cta_first[grid] != p.n_units) {
+            std::printf("FAIL schedule holds %d of %d units\n", (int)p.cta_first[grid], p.n_units);
+            return 1;
+        }
+        std::vector<int> hit(p.n_units, 0);
+        long long total = 0, worst = 0, biggest = 0;
+        for (int c = 0; c < grid; ++c) {
+            long long t = 0;
+            for (int k = p.cta_first[c]; k < p.cta_first[c + 1]; ++k) {
+                const int u = p.sched[k];
+                if (u >= p.n_units || ++hit[u] != 1) {
+                    std::printf("FAIL schedule repeats or exceeds unit %d\n", u);
+                    return 1;
+                }
+                int bh;
+                const long long cost = npa::patch_cost(p, npa::unit_patch(p, u, &bh)) + npa::kUnitOverheadBlocks;
+                t += cost;
+                if (cost > biggest) biggest = cost;
+                if (k == p.cta_first[c]) first_bh.insert(bh);
+            }
+            total += t;
+            if (t > worst) worst = t;
+        }
+        balance = (double)worst * grid / (double)total;
+        bound = 1.0 + (double)biggest * grid / (double)total;  // list scheduling: mean + one unit
+    }
+    std::printf("ok units %d ordered %d classes %d wave_heads %d sched %d balance %.4f first_heads %d bound %.4f\n",
+                p.n_units, p.n_perm, p.n_cls, (int)wave_bh.size(), p.n_sched, balance, (int)first_bh.size(), bound);
     return 0;
 }
