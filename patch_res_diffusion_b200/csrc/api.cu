@@ -100,6 +100,51 @@ npa_status ensure_ready(int *sm_count = nullptr, int *l2_bytes = nullptr) {
     return ds.status;
 }
 
+// The per-CTA unit lists take 0.1-0.5 ms to build on the host, so the last
+// few are kept, keyed by everything they depend on.
+struct SchedKey {
+    int BH, H, W, G, Ph, Pw, mh, mw, kc_log2, kr, n_qblocks, patch_begin, patch_count, grid, head_major;
+    bool operator==(const SchedKey &o) const { return std::memcmp(this, &o, sizeof(SchedKey)) == 0; }
+};
+struct SchedEntry {
+    SchedKey key;
+    unsigned long long used = 0;  // 0: empty
+    int n_sched = 0;
+    unsigned short cta_first[npa::kMaxSchedCtas + 1];
+    unsigned short sched[npa::kMaxSchedUnits];
+};
+constexpr int kSchedCacheEntries = 8;
+std::mutex g_sched_mu;
+SchedEntry g_sched_cache[kSchedCacheEntries];
+unsigned long long g_sched_clock = 0;
+
+// Fills prm's per-CTA lists (npa::build_schedule), from the cache when the
+// same geometry was scheduled recently.
+void schedule_units(FwdParams &prm, int grid, bool head_major) {
+    SchedKey key;
+    std::memset(&key, 0, sizeof(key));
+    key = SchedKey{prm.BH, prm.H,      prm.W,  prm.G,         prm.Ph,          prm.Pw,          prm.mh,          prm.mw,
+                   prm.kc_log2, prm.kr, prm.n_qblocks, prm.patch_begin, prm.patch_count, grid, head_major ? 1 : 0};
+    std::lock_guard<std::mutex> lock(g_sched_mu);
+    SchedEntry *victim = &g_sched_cache[0];
+    for (SchedEntry &e : g_sched_cache) {
+        if (e.used && e.key == key) {
+            e.used = ++g_sched_clock;
+            prm.n_sched = e.n_sched;
+            std::memcpy(prm.cta_first, e.cta_first, sizeof(e.cta_first));
+            std::memcpy(prm.sched, e.sched, sizeof(unsigned short) * (size_t)e.n_sched);
+            return;
+        }
+        if (e.used < victim->used) victim = &e;
+    }
+    npa::build_schedule(prm, grid, head_major);
+    victim->key = key;
+    victim->used = ++g_sched_clock;
+    victim->n_sched = prm.n_sched;
+    std::memcpy(victim->cta_first, prm.cta_first, sizeof(prm.cta_first));
+    std::memcpy(victim->sched, prm.sched, sizeof(unsigned short) * (size_t)prm.n_sched);
+}
+
 // Rectangle form of both geometries (see npa_geometry.cuh).
 struct Geo {
     int H, W, Ph, Pw, mh, mw;
@@ -316,7 +361,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     if (false) {
 #endif
         const double kv_bytes = 4.0 * BH * (double)g.H * g.W * d + 4.0 * BH * (double)G * d;
-        npa::build_schedule(prm, (int)grid, kv_bytes > (double)l2_bytes);
+        schedule_units(prm, (int)grid, kv_bytes > (double)l2_bytes);
     }
     const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)BH};
     const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)g.W * d * 2, (cuuint64_t)g.H * g.W * d * 2};

@@ -1,44 +1,47 @@
 // npa_fwd_kernel.cuh - the sm_100a forward kernel for patch-restricted
 // self-attention (NPA and PCPP share it through npa_geometry.cuh).
 //
-// A persistent CTA works through units of NT query tiles (128 queries each) of
-// one patch that share the patch's key/value window, streamed in blocks of KB
-// keys. Every path runs NT = 2, KB = 128.
-// Warps (NT + 1 warpgroups):
-//   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes 0..127)
-//   control warp 0     TMA producer (Q once per unit, then K and V blocks
-//                      through a ring of kStages shared-memory stages); owns
-//                      the TMEM allocation
+// A persistent CTA works through units of NT = 2 query tiles (128 queries
+// each) of one patch that share the patch's key/value window, streamed in
+// blocks of KB = 128 keys.
+// Warps (NT * kHalves + 1 warpgroups):
+//   warpgroup g < NT * kHalves   softmax + epilogue for query tile g / kHalves,
+//                      score columns and output columns of half g % kHalves
+//                      (TMEM lanes 0..127: one query row per thread)
+//   control warp 0     TMA producer (Q once per unit, double-buffered at
+//                      d = 64, then K and V blocks through a ring of kStages
+//                      shared-memory stages); owns the TMEM allocation
 //   control warp 1     MMA issuer: d = 64, the S = Q K^T products; d = 128, all
 //   control warp 2     d = 64: MMA issuer of the O += P V products
 // The kernel is launched with kRegsLaunch registers per thread; the control
 // warpgroup gives registers back (setmaxnreg.dec to kRegsCtl) and the softmax
-// warpgroups take them (setmaxnreg.inc to kRegsSoftmax), NT * 128 *
-// kRegsSoftmax + 128 * kRegsCtl being the launch's total.
+// warpgroups take them (setmaxnreg.inc to kRegsSoftmax). The host checks the
+// compiled register count before the first launch.
 //
 // Per key block j and tile q the MMA warp issues S_q = Q_q K_j^T into TMEM
 // (M=128, N=KB, K=d, both operands K-major in 128-byte-swizzled shared
-// memory); the softmax warps read S_q from TMEM (one thread per query row),
-// update the running maximum and sum, and write P_q as bf16 into TMEM; the MMA
-// warp then issues O_q += P_q V_j with A = P_q read from TMEM and B = V_j
-// (MN-major, 128-byte swizzle).
+// memory); the softmax warps read S_q from TMEM, update the running maximum
+// and sum, and write P_q as bf16 into TMEM; the MMA warp then issues O_q +=
+// P_q V_j with A = P_q read from TMEM and B = V_j (MN-major, 128-byte swizzle).
 //
-// TMEM (512 columns x 128 lanes). d = 64: S_0..S_{NT-1} | O_0.. | P_0.., so P
+// TMEM (512 columns x 128 lanes). d = 64: S_0 S_1 | O_0 O_1 | P_0 P_1, so P
 // has its own buffer and the MMA warp issues S_q(j+1) as soon as the softmax
 // warps have copied S_q(j) into registers: the softmax runs back to back while
-// the tensor core computes the next scores. d = 128: S0 S1 | O0 O1 with P_q in
-// the first 64 columns of S_q; the MMA warp then issues PV_q(j-1) before
+// the tensor core computes the next scores. d = 128: S0 S1 | O0 O1 with P_q
+// over the first columns of S_q; the MMA warp then issues PV_q(j-1) before
 // S_q(j), and because tcgen05 operations of one thread complete in order, the
 // commit that announces S_q(j) also guarantees that PV_q(j-1) has finished.
 //
-// Softmax arithmetic per block. At d = 64 the softmax warpgroups take turns on
-// the exponential unit (MUFU), round robin, block by block; the turn passes
-// between the warps that share a sub-partition (warp k of each group), so a
-// warp waits only for its own sub-partition's partner: warp k of group q
-// loads its scores and takes the block maximum (a tree of three-input maxima)
-// while its partner evaluates exponentials, then waits for its turn,
-// evaluates its 32 rows x KB exponentials and passes the turn on, so loads,
-// stores and barrier traffic overlap the partner's exponentials.
+// Softmax arithmetic per block. At d = 64 each tile has two warpgroups, one
+// per half of the block's 128 score columns, so on every sub-partition the two
+// warps serving a tile evaluate exponentials at the same time (one warp alone
+// cannot keep the special-function unit busy). They agree on the block
+// maximum through shared memory (and, at the end of a unit, on the row sum),
+// so both take the same decision on the reference. The two tiles take turns
+// on the exponential unit (MUFU), block by block; the turn passes between the
+// warps that share a sub-partition, so a warp waits only for its own
+// sub-partition's partners, and loads, maxima, exchanges and stores overlap
+// the other tile's exponentials.
 // p = 2^(s*log2(e)/sqrt(d) - R) on the packed f32x2 FMA path and
 // ex2.approx.f32, rounded to bf16 pairs for P and summed in float32 (four
 // packed partial sums). The reference R is moved lazily: only when the block
@@ -105,10 +108,13 @@ template <int D, int NT, int KB>
 struct KCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(NT == 2 && KB == 128, "two query tiles per CTA, 128-key blocks");
+#ifndef NPA_D64_HALVES
+#define NPA_D64_HALVES 1
+#endif
 #ifndef NPA_D128_HALVES
 #define NPA_D128_HALVES 1
 #endif
-    static constexpr int kHalves = D == 64 ? 2 : NPA_D128_HALVES;  // softmax warpgroups per query tile
+    static constexpr int kHalves = D == 64 ? NPA_D64_HALVES : NPA_D128_HALVES;  // softmax warpgroups per query tile
     static_assert(kHalves == 1 || kHalves == 2, "column halves");
     static constexpr int kCols = KB / kHalves;              // scores per thread per key block
     static constexpr int kOCols = D / kHalves;              // output columns per thread
@@ -585,16 +591,14 @@ __device__ __forceinline__ void exp2_fma_x2(uint64_t x2, float &p0, float &p1) {
     p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
-// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum
-// returned. POLY > 0: every POLY-th pair on the FMA pipe (no -inf scores).
-template <int KB, int POLY>
-__device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2]) {
-    const float neg = (ref == -INFINITY) ? 0.f : -ref;
-    const uint64_t c2 = sm100::pack_f32x2(c, c);
-    const uint64_t m2 = sm100::pack_f32x2(neg, neg);
-    uint64_t acc[4] = {0, 0, 0, 0};
+// p = 2^(s*c - ref) for the scores of pairs [I0, I1): packed bf16 pairs
+// into pk, float32 partial sums into acc. POLY > 0: every POLY-th pair on the
+// FMA pipe (no -inf scores).
+template <int KB, int POLY, int I0, int I1>
+__device__ __forceinline__ void exp_range(const float (&s)[KB], uint64_t c2, uint64_t m2, uint32_t (&pk)[KB / 2],
+                                          uint64_t (&acc)[4]) {
 #pragma unroll
-    for (int i = 0; i < KB / 2; ++i) {
+    for (int i = I0; i < I1; ++i) {
         const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
         float p0, p1;
         if (POLY > 0 && i % (POLY > 0 ? POLY : 1) == POLY - 1) {
@@ -608,6 +612,27 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
         pk[i] = sm100::pack_bf16x2(p0, p1);
         acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
     }
+}
+
+// Hand-off point of the exponential unit's turn, in pairs before the end of a
+// thread's block (0: after the whole block is issued). Build option.
+#ifndef NPA_TURN_EARLY
+#define NPA_TURN_EARLY 0
+#endif
+
+// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum
+// returned; `handoff` runs after pair KB/2 - NPA_TURN_EARLY has been issued.
+template <int KB, int POLY, typename F>
+__device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2],
+                                           F &&handoff) {
+    const float neg = (ref == -INFINITY) ? 0.f : -ref;
+    const uint64_t c2 = sm100::pack_f32x2(c, c);
+    const uint64_t m2 = sm100::pack_f32x2(neg, neg);
+    uint64_t acc[4] = {0, 0, 0, 0};
+    constexpr int kSplit = KB / 2 - NPA_TURN_EARLY;
+    exp_range<KB, POLY, 0, kSplit>(s, c2, m2, pk, acc);
+    handoff();
+    exp_range<KB, POLY, kSplit, KB / 2>(s, c2, m2, pk, acc);
     float a0, a1, b0, b1, c0, c1, d0, d1;
     sm100::unpack_f32x2(acc[0], a0, a1);
     sm100::unpack_f32x2(acc[1], b0, b1);
@@ -746,17 +771,19 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
             break;
         }
         uint32_t pk[kC / 2];
+        // pass the turn to the next tile's warps on this sub-partition once
+        // the block's exponentials are issued
+        auto handoff = [&]() {
+            if (C::kUseTurn) {
+                __syncwarp();
+                if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
+            }
+        };
         float blk_sum;
         if (kPolyEvery > 0 && C::kSeparateP && !masked)
-            blk_sum = exp_block<kC, (C::kSeparateP ? kPolyEvery : 0)>(s, sl2, R, pk);
+            blk_sum = exp_block<kC, (C::kSeparateP ? kPolyEvery : 0)>(s, sl2, R, pk, handoff);
         else
-            blk_sum = exp_block<kC, 0>(s, sl2, R, pk);
-        // pass the turn to the next tile's warps on this sub-partition once
-        // the whole block is issued
-        if (C::kUseTurn) {
-            __syncwarp();
-            if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
-        }
+            blk_sum = exp_block<kC, 0>(s, sl2, R, pk, handoff);
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
         if (C::kSeparateP && j > w.jb) {
             // PV_q(j-1) must be done before O is rescaled or P_q overwritten
@@ -945,7 +972,7 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
     volatile uint32_t *abort_flag = &misc[1];
 
     if (warp >= C::kCtlWarp) {
-        sm100::setmaxnreg_dec<C::kRegsCtl>();
+        if constexpr (C::kRegsCtl < C::kRegsLaunch) sm100::setmaxnreg_dec<C::kRegsCtl>();
         const int role = warp - C::kCtlWarp;
         if ((threadIdx.x & 31) == 0) {
             if (role == 0) run_producer<D, NT, KB, GQ>(p, smem, bars, abort_flag);
@@ -957,7 +984,7 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
             }
         }
     } else {
-        sm100::setmaxnreg_inc<C::kRegsSoftmax>();
+        if constexpr (C::kRegsSoftmax > C::kRegsLaunch) sm100::setmaxnreg_inc<C::kRegsSoftmax>();
         run_softmax<D, NT, KB, GQ, MD>(p, smem, bars, tmem, abort_flag, warp >> 2);
     }
 

@@ -146,6 +146,12 @@ inline int patch_cost(const FwdParams &p, int patch) {
     return cdiv_(ww, kc) * cdiv_(wh, p.kr);
 }
 
+// Host: the predicted cost of one unit of a patch, in key blocks: its
+// window's blocks, the global-token blocks and kUnitOverheadBlocks.
+inline long long unit_cost(const FwdParams &p, int patch) {
+    return patch_cost(p, patch) + cdiv_(p.G, p.kb) + kUnitOverheadBlocks;
+}
+
 // Host: fills patch_order with the patches [patch_begin, patch_begin +
 // patch_count) by decreasing cost (ties in natural order), so a persistent
 // CTA's last units are its cheapest, and cls_rank0 with the runs of equal
@@ -214,68 +220,149 @@ __host__ __device__ inline int unit_patch(const FwdParams &p, int unit, int *bh)
     return p.n_perm ? int(p.patch_order[rank]) : p.patch_begin + rank;
 }
 
-// Host: the per-CTA unit lists. Units are taken in one global order and each
-// goes to the CTA that becomes free first (list scheduling on the predicted
-// cost: the key blocks of the unit's window plus kUnitOverheadBlocks), so the
-// CTAs finish together and, at any moment, the running units lie close
-// together in the global order. The global order is the unit numbering
-// (cost class, then batch*head, then patch, then query-tile group: cheapest
-// last) or, with head_major, batch*head first and then cost class, patch and
-// query-tile group, so that the units running at one time share one or two
-// heads' keys and values (a whole head's windows stay in L2, instead of being
-// read again for every cost class). Needs order_patches() done with a class
-// table; leaves n_sched = 0 (round robin) otherwise or past the table sizes.
+// Host: the per-CTA unit lists, on the predicted unit costs (unit_cost).
+//  * head_major (the keys and values of all heads do not fit in L2): units
+//    are taken batch*head first, then cost class, patch and query-tile
+//    group, and each goes to the CTA that becomes free first (list
+//    scheduling), so the CTAs finish together and the units running at one
+//    moment share one or two heads' keys and values (a head's windows stay
+//    in L2 instead of being read again for every cost class).
+//  * otherwise (everything fits in L2): the split of every cost class over
+//    the CTAs is chosen for the smallest largest CTA cost - longest units
+//    first, then moves and swaps of single units off the busiest CTA while
+//    they lower it - and each CTA runs its units costliest class first, the
+//    units of a class dealt round robin in the unit numbering.
+// Needs order_patches() done with a class table; leaves n_sched = 0 (round
+// robin) otherwise or past the table sizes.
 inline void build_schedule(FwdParams &p, int grid, bool head_major) {
     p.n_sched = 0;
     if (p.n_cls == 0 || p.n_units > kMaxSchedUnits || grid > kMaxSchedCtas || grid < 1) return;
-    static thread_local unsigned short order[kMaxSchedUnits];
-    static thread_local unsigned short owner[kMaxSchedUnits];
-    int n = 0;
     const int nq = p.n_qblocks;
+    const int ncls = p.n_cls;
+    long long ccost[kMaxCostClasses];
+    for (int k = 0; k < ncls; ++k)
+        ccost[k] = unit_cost(p, p.n_perm ? int(p.patch_order[p.cls_rank0[k]]) : p.patch_begin + p.cls_rank0[k]);
+    long long load[kMaxSchedCtas];
+    int count[kMaxSchedCtas];
+    for (int c = 0; c < grid; ++c) load[c] = count[c] = 0;
     if (head_major) {
+        static thread_local unsigned short order[kMaxSchedUnits];
+        static thread_local unsigned short owner[kMaxSchedUnits];
+        int n = 0;
         for (int bh = 0; bh < p.BH; ++bh)
-            for (int c = 0; c < p.n_cls; ++c) {
+            for (int c = 0; c < ncls; ++c) {
                 const int cnt = p.cls_rank0[c + 1] - p.cls_rank0[c];
                 for (int k = 0; k < cnt; ++k)
                     for (int qb = 0; qb < nq; ++qb)
                         order[n++] = (unsigned short)((p.BH * p.cls_rank0[c] + bh * cnt + k) * nq + qb);
             }
-    } else {
-        for (int u = 0; u < p.n_units; ++u) order[n++] = (unsigned short)u;
+        // binary min-heap of (finish time, cta), ties to the lower CTA index
+        int heap[kMaxSchedCtas];
+        for (int c = 0; c < grid; ++c) heap[c] = c;
+        auto less = [&](int a, int b) { return load[a] < load[b] || (load[a] == load[b] && a < b); };
+        for (int i = 0; i < n; ++i) {
+            int bh;
+            const int c = heap[0];
+            owner[i] = (unsigned short)c;
+            ++count[c];
+            load[c] += unit_cost(p, unit_patch(p, order[i], &bh));
+            for (int k = 0;;) {  // sift the root down
+                const int l = 2 * k + 1, r = l + 1;
+                int m = k;
+                if (l < grid && less(heap[l], heap[m])) m = l;
+                if (r < grid && less(heap[r], heap[m])) m = r;
+                if (m == k) break;
+                const int t = heap[k];
+                heap[k] = heap[m];
+                heap[m] = t;
+                k = m;
+            }
+        }
+        p.cta_first[0] = 0;
+        for (int c = 0; c < grid; ++c) p.cta_first[c + 1] = (unsigned short)(p.cta_first[c] + count[c]);
+        int fill[kMaxSchedCtas];
+        for (int c = 0; c < grid; ++c) fill[c] = p.cta_first[c];
+        for (int i = 0; i < n; ++i) p.sched[fill[owner[i]]++] = order[i];
+        p.n_sched = n;
+        return;
     }
-    // binary min-heap of (finish time, cta), ties to the lower CTA index
-    long long tfin[kMaxSchedCtas];
-    int heap[kMaxSchedCtas], count[kMaxSchedCtas];
-    for (int c = 0; c < grid; ++c) {
-        tfin[c] = 0;
-        heap[c] = c;
-        count[c] = 0;
+    // units of class k: numbers [BH * cls_rank0[k] * nq, BH * cls_rank0[k+1] * nq)
+    static thread_local int cnt[kMaxSchedCtas][kMaxCostClasses];
+    for (int c = 0; c < grid; ++c)
+        for (int k = 0; k < ncls; ++k) cnt[c][k] = 0;
+    for (int k = 0; k < ncls; ++k) {  // longest units first, each to the least loaded CTA
+        const int units_k = p.BH * (p.cls_rank0[k + 1] - p.cls_rank0[k]) * nq;
+        for (int i = 0; i < units_k; ++i) {
+            int c = 0;
+            for (int d = 1; d < grid; ++d)
+                if (load[d] < load[c]) c = d;
+            ++cnt[c][k];
+            load[c] += ccost[k];
+        }
     }
-    auto less = [&](int a, int b) { return tfin[a] < tfin[b] || (tfin[a] == tfin[b] && a < b); };
-    for (int i = 0; i < n; ++i) {
-        int bh;
-        const int c = heap[0];
-        owner[i] = (unsigned short)c;
-        ++count[c];
-        tfin[c] += patch_cost(p, unit_patch(p, order[i], &bh)) + kUnitOverheadBlocks;
-        for (int k = 0;;) {  // sift the root down
-            const int l = 2 * k + 1, r = l + 1;
-            int m = k;
-            if (l < grid && less(heap[l], heap[m])) m = l;
-            if (r < grid && less(heap[r], heap[m])) m = r;
-            if (m == k) break;
-            const int t = heap[k];
-            heap[k] = heap[m];
-            heap[m] = t;
-            k = m;
+    for (int it = 0; it < 64 * grid; ++it) {  // improve the busiest CTA while possible
+        int cm = 0;
+        for (int d = 1; d < grid; ++d)
+            if (load[d] > load[cm]) cm = d;
+        long long best = load[cm];
+        int bk = -1, bc = -1, bm = -1;  // class moved off cm, receiving CTA, class moved back (-1: none)
+        for (int k = 0; k < ncls; ++k) {
+            if (!cnt[cm][k]) continue;
+            for (int c = 0; c < grid; ++c) {
+                if (c == cm) continue;
+                const long long mv = load[c] + ccost[k] > load[cm] - ccost[k] ? load[c] + ccost[k] : load[cm] - ccost[k];
+                if (mv < best) {
+                    best = mv;
+                    bk = k;
+                    bc = c;
+                    bm = -1;
+                }
+                for (int m = 0; m < ncls; ++m) {
+                    if (!cnt[c][m] || ccost[m] >= ccost[k]) continue;
+                    const long long a = load[cm] - ccost[k] + ccost[m], b2 = load[c] + ccost[k] - ccost[m];
+                    const long long sw = a > b2 ? a : b2;
+                    if (sw < best) {
+                        best = sw;
+                        bk = k;
+                        bc = c;
+                        bm = m;
+                    }
+                }
+            }
+        }
+        if (bk < 0) break;
+        --cnt[cm][bk];
+        ++cnt[bc][bk];
+        load[cm] -= ccost[bk];
+        load[bc] += ccost[bk];
+        if (bm >= 0) {
+            --cnt[bc][bm];
+            ++cnt[cm][bm];
+            load[bc] -= ccost[bm];
+            load[cm] += ccost[bm];
         }
     }
     p.cta_first[0] = 0;
-    for (int c = 0; c < grid; ++c) p.cta_first[c + 1] = (unsigned short)(p.cta_first[c] + count[c]);
+    for (int c = 0; c < grid; ++c) {
+        int t = 0;
+        for (int k = 0; k < ncls; ++k) t += cnt[c][k];
+        p.cta_first[c + 1] = (unsigned short)(p.cta_first[c] + t);
+    }
     int fill[kMaxSchedCtas];
     for (int c = 0; c < grid; ++c) fill[c] = p.cta_first[c];
-    for (int i = 0; i < n; ++i) p.sched[fill[owner[i]]++] = order[i];
-    p.n_sched = n;
+    for (int k = 0; k < ncls; ++k) {  // deal class k's units round robin to the CTAs that take some
+        int left[kMaxSchedCtas];
+        for (int c = 0; c < grid; ++c) left[c] = cnt[c][k];
+        const int u0 = p.BH * p.cls_rank0[k] * nq, u1 = p.BH * p.cls_rank0[k + 1] * nq;
+        int c = 0;
+        for (int u = u0; u < u1; ++u) {
+            while (left[c] == 0) c = c + 1 == grid ? 0 : c + 1;
+            p.sched[fill[c]++] = (unsigned short)u;
+            --left[c];
+            c = c + 1 == grid ? 0 : c + 1;
+        }
+    }
+    p.n_sched = p.n_units;
 }
 
 // The i-th unit of this CTA's work, or -1 past its last.

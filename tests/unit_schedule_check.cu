@@ -122,7 +122,7 @@ int main(int argc, char **argv) {
                     return 1;
                 }
                 int bh;
-                const long long cost = npa::patch_cost(p, npa::unit_patch(p, u, &bh)) + npa::kUnitOverheadBlocks;
+                const long long cost = npa::unit_cost(p, npa::unit_patch(p, u, &bh));
                 t += cost;
                 if (cost > biggest) biggest = cost;
                 if (k == p.cta_first[c]) first_bh.insert(bh);
