@@ -4,10 +4,9 @@
 // A persistent CTA works through units of NT = 2 query tiles (128 queries
 // each) of one patch that share the patch's key/value window, streamed in
 // blocks of KB = 128 keys.
-// Warps (NT * kHalves + 1 warpgroups):
-//   warpgroup g < NT * kHalves   softmax + epilogue for query tile g / kHalves,
-//                      score columns and output columns of half g % kHalves
-//                      (TMEM lanes 0..127: one query row per thread)
+// Warps (NT + 1 warpgroups):
+//   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes
+//                      0..127: one query row per thread)
 //   control warp 0     TMA producer (Q once per unit, double-buffered at
 //                      d = 64, then K and V blocks through a ring of kStages
 //                      shared-memory stages); owns the TMEM allocation
@@ -32,16 +31,14 @@
 // S_q(j), and because tcgen05 operations of one thread complete in order, the
 // commit that announces S_q(j) also guarantees that PV_q(j-1) has finished.
 //
-// Softmax arithmetic per block. At d = 64 each tile has two warpgroups, one
-// per half of the block's 128 score columns, so on every sub-partition the two
-// warps serving a tile evaluate exponentials at the same time (one warp alone
-// cannot keep the special-function unit busy). They agree on the block
-// maximum through shared memory (and, at the end of a unit, on the row sum),
-// so both take the same decision on the reference. The two tiles take turns
-// on the exponential unit (MUFU), block by block; the turn passes between the
-// warps that share a sub-partition, so a warp waits only for its own
-// sub-partition's partners, and loads, maxima, exchanges and stores overlap
-// the other tile's exponentials.
+// Softmax arithmetic per block. At d = 64 the softmax warpgroups take turns on
+// the exponential unit (MUFU), round robin, block by block; the turn passes
+// between the warps that share a sub-partition (warp k of each group), so a
+// warp waits only for its own sub-partition's partner: warp k of group q
+// loads its scores and takes the block maximum (a tree of three-input maxima)
+// while its partner evaluates exponentials, then waits for its turn,
+// evaluates its 32 rows x KB exponentials and passes the turn on, so loads,
+// stores and barrier traffic overlap the partner's exponentials.
 // p = 2^(s*log2(e)/sqrt(d) - R) on the packed f32x2 FMA path and
 // ex2.approx.f32, rounded to bf16 pairs for P and summed in float32 (four
 // packed partial sums). The reference R is moved lazily: only when the block
@@ -97,28 +94,13 @@ __device__ __forceinline__ bool bound_row(bool valid, size_t row, size_t rows) {
 
 constexpr float kRescaleLog2 = 8.0f;  // lazy rescale threshold (log2 units)
 
-// Kernel shape: D = head dimension, NT = query tiles per CTA, KB = keys per
-// key block. At d = 64 every query tile has two softmax warpgroups, one per
-// half of the block's score columns (kHalves = 2): the two warps of a
-// sub-partition that serve one tile evaluate their exponentials at the same
-// time, which keeps the exponential unit busier than one warp can, and they
-// agree on the block maximum (and at the end on the row sum) through a small
-// shared-memory exchange. At d = 128 one warpgroup serves a tile.
+// Kernel shape: D = head dimension, NT = query tiles per CTA (one softmax
+// warpgroup each), KB = keys per key block.
 template <int D, int NT, int KB>
 struct KCfg {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(NT == 2 && KB == 128, "two query tiles per CTA, 128-key blocks");
-#ifndef NPA_D64_HALVES
-#define NPA_D64_HALVES 1
-#endif
-#ifndef NPA_D128_HALVES
-#define NPA_D128_HALVES 1
-#endif
-    static constexpr int kHalves = D == 64 ? NPA_D64_HALVES : NPA_D128_HALVES;  // softmax warpgroups per query tile
-    static_assert(kHalves == 1 || kHalves == 2, "column halves");
-    static constexpr int kCols = KB / kHalves;              // scores per thread per key block
-    static constexpr int kOCols = D / kHalves;              // output columns per thread
-    static constexpr int kSoftmaxWGs = NT * kHalves;
+    static constexpr int kSoftmaxWGs = NT;
     static constexpr int kChunks = D / 64;                 // 64-element (128-byte) column blocks
     static constexpr int kQChunkBytes = 128 * 128;         // 128 query rows x 128 bytes
     static constexpr int kQTileBytes = kChunks * kQChunkBytes;
@@ -132,9 +114,9 @@ struct KCfg {
     // since a split above the launch total would never complete), then after
     // the control warpgroup gives registers back and the softmax warpgroups
     // take them
-    static constexpr uint32_t kRegsLaunch = kHalves == 2 ? 96 : 168;
-    static constexpr uint32_t kRegsSoftmax = kHalves == 1 ? 216 : (D == 64 ? 104 : 96);
-    static constexpr uint32_t kRegsCtl = kHalves == 1 ? 72 : (D == 64 ? 64 : 96);
+    static constexpr uint32_t kRegsLaunch = 168;
+    static constexpr uint32_t kRegsSoftmax = 216;
+    static constexpr uint32_t kRegsCtl = 72;
     static_assert(kSoftmaxWGs * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
     static_assert(kThreads * kRegsLaunch <= 65536, "register file");
     // query buffers: at d = 64 two, so that the next unit's tiles load while
@@ -156,29 +138,23 @@ struct KCfg {
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
     static constexpr int bSFull = bVEmpty + kStages;   // [NT] S_q written (MMA commit)
-    static constexpr int bSFree = bSFull + NT;         // [NT] S_q copied to registers (128 * kHalves arrivals)
-    static constexpr int bPFull = bSFree + NT;         // [NT] P_q written (128 * kHalves arrivals)
+    static constexpr int bSFree = bSFull + NT;         // [NT] S_q copied to registers (128 arrivals)
+    static constexpr int bPFull = bSFree + NT;         // [NT] P_q written (128 arrivals)
     static constexpr int bPFree = bPFull + NT;         // [NT] PV_q done (MMA commit)
-    // [NT][4] exponential-phase turn of warp k of tile q's warpgroups (one
-    // arrival per warpgroup of the tile): the turn passes between the warps
-    // that share a sub-partition's MUFU
+    // [NT][4] exponential-phase turn of warp k of warpgroup q (1 arrival): the
+    // turn passes between the warps that share a sub-partition's MUFU
     static constexpr int bTurn = bPFree + NT;
     static constexpr int bDrain = bTurn + 4 * NT;      // [2] one per MMA-issuing warp
-    // [NT][4] (kHalves == 2) exchange between warp k of the two warpgroups of
-    // tile q (64 arrivals): block maxima, then the row sums
-    static constexpr int bXchg = bDrain + 2;
-    static constexpr int kNumBars = bXchg + 4 * NT;
+    static constexpr int kNumBars = bDrain + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-    static constexpr int kOffXchg = kOffMisc + 16;     // float [NT][kHalves][2 parities][128 rows]
-    static constexpr int kXchgBytes = kHalves == 2 ? NT * 2 * 2 * 128 * 4 : 0;
-    static constexpr int kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + slack for 1024-byte alignment
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
     static_assert(kSmemBytes <= 227 * 1024, "shared memory");
     // tensor memory columns
     static constexpr uint32_t kTmemCols = 512;
     static constexpr bool kSeparateP = (D == 64);
-    // d = 64: the tiles' warpgroup pairs hand the exponential unit to each
-    // other in turn; d = 128: the aliased-P issue order already alternates the
-    // tiles and the hand-off costs about 3%.
+    // d = 64: the softmax warpgroups hand the exponential unit to each other
+    // in turn; d = 128: the aliased-P issue order already alternates the tiles
+    // and the hand-off costs about 3%.
 #ifndef NPA_D64_TURN
 #define NPA_D64_TURN 1
 #endif
@@ -187,13 +163,6 @@ struct KCfg {
     __device__ static constexpr uint32_t col_o(int q) { return uint32_t(NT * KB + q * D); }
     __device__ static constexpr uint32_t col_p(int q) {
         return kSeparateP ? uint32_t(NT * KB + NT * D + q * (KB / 2)) : col_s(q);
-    }
-    // P of column half h (keys [h * kCols, (h + 1) * kCols), packed bf16
-    // pairs: kCols / 2 columns): d = 64 in the separate P buffer, one after
-    // the other; d = 128 over the first columns of that half's own scores
-    // (which its warps have already read)
-    __device__ static constexpr uint32_t col_p_half(int q, int h) {
-        return kSeparateP ? col_p(q) + uint32_t(h * (kCols / 2)) : col_s(q) + uint32_t(h * kCols);
     }
     static_assert(!kSeparateP || NT * KB + NT * D + NT * (KB / 2) <= 512, "tensor memory columns");
     static_assert(kSeparateP || NT * KB + NT * D <= 512, "tensor memory columns");
@@ -355,11 +324,10 @@ template <int D, int NT, int KB>
 __device__ __forceinline__ void issue_pv(uint32_t tmem, int q, uint64_t vdesc, bool accumulate) {
     using C = KCfg<D, NT, KB>;
     constexpr uint32_t kIdO = sm100::idesc_bf16_f32(128, D, false, true);  // O += P V, V MN-major
-    constexpr int kStepsPerHalf = C::kCols / 16;  // K16 steps per column half of P
 #pragma unroll
     for (int kk = 0; kk < KB / 16; ++kk)
-        sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p_half(q, kk / kStepsPerHalf) + (kk % kStepsPerHalf) * 8,
-                      vdesc + uint64_t((kk * 2048) >> 4), kIdO, (accumulate || kk > 0) ? 1u : 0u);
+        sm100::mma_ts(tmem + C::col_o(q), tmem + C::col_p(q) + kk * 8, vdesc + uint64_t((kk * 2048) >> 4), kIdO,
+                      (accumulate || kk > 0) ? 1u : 0u);
 }
 
 struct OperandDescs {
@@ -641,45 +609,24 @@ __device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float 
     return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
-// Exchange between the two warps (one per column half) that serve the same
-// 32 rows of a query tile: each writes its value for its row, arrives on the
-// pair's barrier (release) and, once the phase completes (acquire), reads the
-// partner's. Slots alternate by phase parity, so a partner one phase ahead
-// cannot overwrite a value before it is read. False if the wait ran out.
-__device__ __forceinline__ bool pair_exchange(float *xbuf, uint64_t *bar, int h, int row, int xp, float mine,
-                                              float &other, uint64_t lim) {
-    const int par = xp & 1;
-    xbuf[(h * 2 + par) * 128 + row] = mine;
-    sm100::mbar_arrive(bar);
-    if (!warp_wait(bar, par, lim)) return false;
-    other = xbuf[((1 - h) * 2 + par) * 128 + row];
-    return true;
-}
-
-// Softmax and epilogue of softmax warpgroup g: query tile q = g / kHalves,
-// score columns [h * kCols, (h + 1) * kCols) of every key block and output
-// columns [h * kOCols, (h + 1) * kOCols), h = g % kHalves. Each thread owns one
-// query row (its TMEM lane).
+// Softmax and epilogue of softmax warpgroup q (query tile q). Each thread owns
+// one query row (its TMEM lane).
 template <int D, int NT, int KB, bool GQ, bool MD>
-__device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint32_t tmem,
-                            volatile uint32_t *abort_flag, int g) {
+__device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, volatile uint32_t *abort_flag,
+                            int q) {
     using C = KCfg<D, NT, KB>;
-    constexpr int kC = C::kCols;
-    const int q = g / C::kHalves, h = g % C::kHalves;
+    constexpr int kC = KB;
     const uint64_t lim = p.wait_limit_ns;
     const int row = threadIdx.x & 127;
     const bool lane0 = (threadIdx.x & 31) == 0;
     const int warp_in_group = (threadIdx.x >> 5) & 3;
     const uint32_t lane_off = uint32_t(warp_in_group) * 32u << 16;
-    const uint32_t tS = tmem + lane_off + C::col_s(q) + uint32_t(h * kC);
-    const uint32_t tO = tmem + lane_off + C::col_o(q) + uint32_t(h * C::kOCols);
-    const uint32_t tP = tmem + lane_off + C::col_p_half(q, h);
-    float *xbuf = reinterpret_cast<float *>(smem + C::kOffXchg) + q * (2 * 2 * 128);
-    uint64_t *xbar = &bars[C::bXchg + 4 * q + warp_in_group];
+    const uint32_t tS = tmem + lane_off + C::col_s(q);
+    const uint32_t tO = tmem + lane_off + C::col_o(q);
+    const uint32_t tP = tmem + lane_off + C::col_p(q);
     const float sl2 = p.scale_log2;
     const int kc = 1 << p.kc_log2;
     int gb = 0;  // global index (across units) of the current block
-    int xp = 0;  // exchange phases completed by this warp pair
     bool ok = true;
     for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
     const Work w = decode<GQ>(p, unit);
@@ -694,7 +641,7 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
     }
     float R = -INFINITY;       // reference maximum (log2 units) of the current block's P
     float R_prev = -INFINITY;  // reference that O and l are currently expressed in
-    float l = 0.f;             // this column half's share of the row sum
+    float l = 0.f;
     for (int j = w.jb; j < w.je; ++j, ++gb) {
         if (!warp_wait(&bars[C::bSFull + q], gb & 1, lim)) {
             ok = false;
@@ -717,19 +664,16 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
             sm100::mbar_arrive(&bars[C::bSFree + q]);
         }
         // keys of this block outside its row segment or the window (or past
-        // the last global token) get -inf; this half's key i is block key
-        // h * kC + i
-        bool masked = false;  // some key of this block (either half) is outside its set
+        // the last global token) get -inf
+        bool masked = false;  // some key of this block is outside its set
         if (j < w.n_win) {
             const int vc = w.wc1 - (w.wc0 + (btc << p.kc_log2));
             const int vr = bend - brow;
             masked = vc < kc || vr < p.kr;
             if (masked) {
 #pragma unroll
-                for (int i = 0; i < kC; ++i) {
-                    const int key = h * kC + i;
-                    if ((key & (kc - 1)) >= vc || (key >> p.kc_log2) >= vr) s[i] = -INFINITY;
-                }
+                for (int i = 0; i < kC; ++i)
+                    if ((i & (kc - 1)) >= vc || (i >> p.kc_log2) >= vr) s[i] = -INFINITY;
             }
             if (++btc == w.wtc) {
                 btc = 0;
@@ -740,39 +684,30 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
                 }
             }
         } else {
-            const int vg = p.G - (j - w.n_win) * KB - h * kC;
-            masked = p.G - (j - w.n_win) * KB < KB;
+            const int vg = p.G - (j - w.n_win) * KB;
+            masked = vg < KB;
             if (vg < kC) {
 #pragma unroll
                 for (int i = 0; i < kC; ++i)
                     if (i >= vg) s[i] = -INFINITY;
             }
         }
-        // block maximum over both column halves, and the reference for this
-        // block's P (lazy: the reference moves only when the maximum grows by
-        // more than kRescaleLog2); both halves take the same decision
-        float bmax = row_max<kC>(s);
-        if constexpr (C::kHalves == 2) {
-            float other;
-            if (!pair_exchange(xbuf, xbar, h, row, xp, bmax, other, lim)) {
-                ok = false;
-                break;
-            }
-            ++xp;
-            bmax = fmaxf(bmax, other);
-        }
-        const float bm = bmax * sl2;
+        // block maximum and the reference for this block's P (lazy: the
+        // reference moves only when the maximum grows by more than
+        // kRescaleLog2)
+        const float bm = row_max<kC>(s) * sl2;
         if (bm > R + kRescaleLog2) R = bm;
-        // wait for this tile's turn on the exponential unit (the turn goes
-        // round the tiles in order, block by block)
+        // wait for this warpgroup's turn on the exponential unit (the turn goes
+        // round the warpgroups in order, block by block)
         if (C::kUseTurn && (q > 0 || gb > 0) &&
             !warp_wait(&bars[C::bTurn + 4 * q + warp_in_group], (q == 0 ? gb - 1 : gb) & 1, lim)) {
             ok = false;
             break;
         }
         uint32_t pk[kC / 2];
-        // pass the turn to the next tile's warps on this sub-partition once
-        // the block's exponentials are issued
+        // pass the turn to the next warpgroup's warp on this sub-partition once
+        // the block's exponentials are issued (handing it over at 3/4 or 7/8
+        // of the block measured 16-17% slower)
         auto handoff = [&]() {
             if (C::kUseTurn) {
                 __syncwarp();
@@ -795,7 +730,7 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
         }
         if (j > w.jb && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-            for (int c = 0; c < C::kOCols / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
 #pragma unroll
@@ -804,10 +739,7 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
             }
         }
         l = l * alpha + blk_sum;
-        if constexpr (kC == 128)
-            sm100::tmem_st64(tP, pk);
-        else
-            sm100::tmem_st32(tP, pk);
+        sm100::tmem_st64(tP, pk);
         sm100::tc_fence_before();
 #ifdef NPA_DEBUG_BOUNDS
         // abort-path test: the last tile of CTA 0 never announces its second
@@ -822,21 +754,9 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
     if (ok && !warp_wait(&bars[C::bPFree + q], (gb - 1) & 1, lim)) ok = false;
     if (!ok) break;
     sm100::tc_fence_after();
-    // the row sum over both column halves, added in the same order by both
-    if constexpr (C::kHalves == 2) {
-        float other;
-        if (!pair_exchange(xbuf, xbar, h, row, xp, l, other, lim)) {
-            ok = false;
-            break;
-        }
-        ++xp;
-        l = h == 0 ? l + other : other + l;
-    }
-    // epilogue: O / l -> bf16 -> the query's token position (this half's
-    // output columns)
+    // epilogue: O / l -> bf16 -> the query's token position
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const int t = w.tile0 + q;
-    const int c0 = h * C::kOCols;
     bool valid;
     size_t out_row;
     if (GQ) {
@@ -847,9 +767,9 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
             // a key-range split: unnormalised O with its reference maximum and row sum
             const size_t prow = (size_t)w.split * p.BH * p.G + out_row;
             valid = bound_row(valid, prow, (size_t)p.n_splits * p.BH * p.G);
-            float4 *part = reinterpret_cast<float4 *>(p.o_part + prow * D + c0);
+            float4 *part = reinterpret_cast<float4 *>(p.o_part + prow * D);
 #pragma unroll
-            for (int c = 0; c < C::kOCols / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
                 if (valid) {
@@ -859,7 +779,7 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
                                                       __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
                 }
             }
-            if (valid && h == 0) *reinterpret_cast<float2 *>(p.ml + prow * 2) = make_float2(R_prev, l);
+            if (valid) *reinterpret_cast<float2 *>(p.ml + prow * 2) = make_float2(R_prev, l);
             continue;
         }
     } else {
@@ -878,9 +798,9 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
             const int cw = md_axis_offset(p.W, p.Pw, p.mw, patch % p.nPw);
             const size_t prow = ((size_t)w.bh * p.md_rows + (rh + grow - w.wr0)) * p.md_tw + (cw + gcol - w.wc0);
             valid = bound_row(valid, prow, (size_t)p.BH * p.md_rows * p.md_tw);
-            float4 *part = reinterpret_cast<float4 *>(p.md_part + prow * D + c0);
+            float4 *part = reinterpret_cast<float4 *>(p.md_part + prow * D);
 #pragma unroll
-            for (int c = 0; c < C::kOCols / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 sm100::tmem_ld32(tO + c * 32, o);
                 if (valid) {
@@ -895,9 +815,9 @@ __device__ void run_softmax(const FwdParams &p, uint8_t *smem, uint64_t *bars, u
         }
     }
     valid = bound_row(valid, out_row, GQ ? (size_t)p.BH * p.G : (size_t)p.BH * p.H * p.W);
-    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D + c0);
+    uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.o) + out_row * D);
 #pragma unroll
-    for (int c = 0; c < C::kOCols / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         sm100::tmem_ld32(tO + c * 32, o);
         if (valid) {
@@ -948,13 +868,10 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
         }
         for (int q = 0; q < NT; ++q) {
             sm100::mbar_init(&bars[C::bSFull + q], 1);
-            sm100::mbar_init(&bars[C::bSFree + q], 128 * C::kHalves);
-            sm100::mbar_init(&bars[C::bPFull + q], 128 * C::kHalves);
+            sm100::mbar_init(&bars[C::bSFree + q], 128);
+            sm100::mbar_init(&bars[C::bPFull + q], 128);
             sm100::mbar_init(&bars[C::bPFree + q], 1);
-            for (int k = 0; k < 4; ++k) {
-                sm100::mbar_init(&bars[C::bTurn + 4 * q + k], C::kHalves);
-                sm100::mbar_init(&bars[C::bXchg + 4 * q + k], 64);  // used when kHalves == 2
-            }
+            for (int k = 0; k < 4; ++k) sm100::mbar_init(&bars[C::bTurn + 4 * q + k], 1);
         }
         sm100::mbar_init(&bars[C::bDrain], 1);
         sm100::mbar_init(&bars[C::bDrain + 1], 1);
@@ -972,7 +889,7 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
     volatile uint32_t *abort_flag = &misc[1];
 
     if (warp >= C::kCtlWarp) {
-        if constexpr (C::kRegsCtl < C::kRegsLaunch) sm100::setmaxnreg_dec<C::kRegsCtl>();
+        sm100::setmaxnreg_dec<C::kRegsCtl>();
         const int role = warp - C::kCtlWarp;
         if ((threadIdx.x & 31) == 0) {
             if (role == 0) run_producer<D, NT, KB, GQ>(p, smem, bars, abort_flag);
@@ -984,8 +901,8 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
             }
         }
     } else {
-        if constexpr (C::kRegsSoftmax > C::kRegsLaunch) sm100::setmaxnreg_inc<C::kRegsSoftmax>();
-        run_softmax<D, NT, KB, GQ, MD>(p, smem, bars, tmem, abort_flag, warp >> 2);
+        sm100::setmaxnreg_inc<C::kRegsSoftmax>();
+        run_softmax<D, NT, KB, GQ, MD>(p, bars, tmem, abort_flag, warp >> 2);
     }
 
     sm100::tc_fence_before();
