@@ -355,11 +355,7 @@ npa_status launch(const void *q, const void *k, const void *v, const void *ks, c
     // gridDim.x-th unit); when the keys and values of all heads do not fit in
     // L2, the lists run head by head
     const unsigned grid = (unsigned)(units < sm_count ? units : sm_count);
-#ifndef NPA_NO_SCHED_LISTS
     if (!md_part) {
-#else
-    if (false) {
-#endif
         const double kv_bytes = 4.0 * BH * (double)g.H * g.W * d + 4.0 * BH * (double)G * d;
         schedule_units(prm, (int)grid, kv_bytes > (double)l2_bytes);
     }

@@ -7,9 +7,9 @@
 // Warps (NT + 1 warpgroups):
 //   warpgroup q < NT   softmax + epilogue for query tile q (TMEM lanes
 //                      0..127: one query row per thread)
-//   control warp 0     TMA producer (Q once per unit, double-buffered at
-//                      d = 64, then K and V blocks through a ring of kStages
-//                      shared-memory stages); owns the TMEM allocation
+//   control warp 0     TMA producer (Q once per unit, then K and V blocks
+//                      through a ring of kStages shared-memory stages); owns
+//                      the TMEM allocation
 //   control warp 1     MMA issuer: d = 64, the S = Q K^T products; d = 128, all
 //   control warp 2     d = 64: MMA issuer of the O += P V products
 // The kernel is launched with kRegsLaunch registers per thread; the control
@@ -106,7 +106,10 @@ struct KCfg {
     static constexpr int kQTileBytes = kChunks * kQChunkBytes;
     static constexpr int kKVChunkBytes = KB * 128;         // KB key rows x 128 bytes
     static constexpr int kKVTileBytes = kChunks * kKVChunkBytes;
-    static constexpr int kStages = D == 128 ? 2 : 4;
+#ifndef NPA_D64_STAGES
+#define NPA_D64_STAGES 4
+#endif
+    static constexpr int kStages = D == 128 ? 2 : NPA_D64_STAGES;
     static constexpr int kThreads = 128 * (kSoftmaxWGs + 1);
     static constexpr int kCtlWarp = 4 * kSoftmaxWGs;       // first warp of the control warpgroup
     // registers per thread: at launch (the most __launch_bounds__ allows for
@@ -119,21 +122,14 @@ struct KCfg {
     static constexpr uint32_t kRegsCtl = 72;
     static_assert(kSoftmaxWGs * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
     static_assert(kThreads * kRegsLaunch <= 65536, "register file");
-    // query buffers: at d = 64 two, so that the next unit's tiles load while
-    // the current unit runs (at d = 128 one: shared memory is full)
-#ifndef NPA_Q_BUFS
-#define NPA_Q_BUFS 2
-#endif
-    static constexpr int kQBufs = D == 64 ? NPA_Q_BUFS : 1;
-    static constexpr int kQBufBytes = NT * kQTileBytes;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kQBufs * kQBufBytes;
+    static constexpr int kOffK = NT * kQTileBytes;
     static constexpr int kOffV = kOffK + kStages * kKVTileBytes;
     static constexpr int kOffBar = kOffV + kStages * kKVTileBytes;
     // barrier indices
-    static constexpr int bQFull = 0;                   // [kQBufs] query tiles landed
-    static constexpr int bQEmpty = bQFull + kQBufs;    // [kQBufs] buffer free (S issuer commit after a unit)
-    static constexpr int bKFull = bQEmpty + kQBufs;
+    static constexpr int bQFull = 0;                   // query tiles landed
+    static constexpr int bQEmpty = 1;                  // Q buffer free (S issuer commit after a unit)
+    static constexpr int bKFull = 2;
     static constexpr int bKEmpty = bKFull + kStages;
     static constexpr int bVFull = bKEmpty + kStages;
     static constexpr int bVEmpty = bVFull + kStages;
@@ -155,10 +151,7 @@ struct KCfg {
     // d = 64: the softmax warpgroups hand the exponential unit to each other
     // in turn; d = 128: the aliased-P issue order already alternates the tiles
     // and the hand-off costs about 3%.
-#ifndef NPA_D64_TURN
-#define NPA_D64_TURN 1
-#endif
-    static constexpr bool kUseTurn = (D == 64) && NPA_D64_TURN;
+    static constexpr bool kUseTurn = (D == 64);
     __device__ static constexpr uint32_t col_s(int q) { return uint32_t(q * KB); }
     __device__ static constexpr uint32_t col_o(int q) { return uint32_t(NT * KB + q * D); }
     __device__ static constexpr uint32_t col_p(int q) {
@@ -231,13 +224,11 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
         // the previous unit's last S products must be done with the Q buffer
-        const int qbuf = uq % C::kQBufs, quse = uq / C::kQBufs;
-        uint8_t *qdst = smem + C::kOffQ + qbuf * C::kQBufBytes;
-        if (quse > 0 && !sm100::mbar_wait(&bars[C::bQEmpty + qbuf], (quse - 1) & 1, lim)) {
+        if (uq > 0 && !sm100::mbar_wait(&bars[C::bQEmpty], (uq - 1) & 1, lim)) {
             ok = false;
             break;
         }
-        sm100::mbar_arrive_expect_tx(&bars[C::bQFull + qbuf], NT * q_bytes);
+        sm100::mbar_arrive_expect_tx(&bars[C::bQFull], NT * q_bytes);
         // a unit's query tile past the patch's last (its outputs are not
         // stored) loads the unit's first tile again, so every box starts
         // inside the tensor
@@ -249,8 +240,8 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
                 const int g0 = bound_coord(tq * 128, p.G);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_3d(qdst + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_gq,
-                                       &bars[C::bQFull + qbuf], c * 64, g0, bh);
+                    sm100::tma_load_3d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_gq,
+                                       &bars[C::bQFull], c * 64, g0, bh);
             } else {
                 int row0, col0;
                 q_tile_origin(p, w, q_tile_valid(p, w, w.tile0 + t) ? w.tile0 + t : w.tile0, &row0, &col0);
@@ -258,8 +249,8 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
                 col0 = bound_coord(col0, p.W);
 #pragma unroll
                 for (int c = 0; c < C::kChunks; ++c)
-                    sm100::tma_load_4d(qdst + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_q,
-                                       &bars[C::bQFull + qbuf], c * 64, col0, row0, bh);
+                    sm100::tma_load_4d(smem + C::kOffQ + t * C::kQTileBytes + c * C::kQChunkBytes, &p.tm_q,
+                                       &bars[C::bQFull], c * 64, col0, row0, bh);
             }
         }
         ++uq;
@@ -291,10 +282,7 @@ __device__ void run_producer(const FwdParams &p, uint8_t *smem, uint64_t *bars, 
     }
     // Drain: every issued copy must have landed before the CTA may exit
     // (immediate on the normal path, where the consumers already saw them).
-    for (int b = 0; b < C::kQBufs && b < uq; ++b) {  // the last unit that used buffer b
-        const int u_last = uq - 1 - ((uq - 1 - b) % C::kQBufs);
-        sm100::mbar_wait(&bars[C::bQFull + b], (u_last / C::kQBufs) & 1, lim);
-    }
+    if (uq > 0) sm100::mbar_wait(&bars[C::bQFull], (uq - 1) & 1, lim);
     for (int s = 0; s < C::kStages; ++s) {
         if (nk > s) sm100::mbar_wait(&bars[C::bKFull + s], ((nk - 1 - s) / C::kStages) & 1, lim);
         if (nv > s) sm100::mbar_wait(&bars[C::bVFull + s], ((nv - 1 - s) / C::kStages) & 1, lim);
@@ -333,7 +321,6 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem, int q, uint64_t vdesc, b
 struct OperandDescs {
     uint64_t q0, k0, v0;  // Q tile 0, K and V stage 0
     uint64_t qtile;       // descriptor increment from one Q tile to the next
-    uint64_t qbuf;        // descriptor increment from one Q buffer to the next
     uint64_t stage;       // descriptor increment from one K/V stage to the next
 };
 
@@ -347,7 +334,6 @@ __device__ __forceinline__ OperandDescs make_descs(uint8_t *smem) {
     d.k0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffK), 16, 1024);
     d.v0 = sm100::sdesc_sw128(sm100::smem_u32(smem + C::kOffV), C::kKVChunkBytes, 1024);
     d.qtile = uint64_t(C::kQTileBytes >> 4);
-    d.qbuf = uint64_t(C::kQBufBytes >> 4);
     d.stage = uint64_t(C::kKVTileBytes >> 4);
     return d;
 }
@@ -368,10 +354,8 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
     for (int ui = 0, unit; ok && (unit = cta_unit(p, ui)) >= 0; ++ui) {
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
-        const int qbuf = uq % C::kQBufs;
-        ok = sm100::mbar_wait(&bars[C::bQFull + qbuf], (uq / C::kQBufs) & 1, lim);
+        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
-        const uint64_t qd = dd.q0 + qbuf * dd.qbuf;
         for (int j = w.jb; ok && j < w.je; ++j, ++gb) {
             if (*abort_flag) {
                 ok = false;
@@ -383,12 +367,12 @@ __device__ void run_mma_s(const FwdParams &p, uint8_t *smem, uint64_t *bars, uin
                 if (gb > 0) ok = sm100::mbar_wait(&bars[C::bSFree + q], (gb - 1) & 1, lim);
                 if (!ok) break;
                 sm100::tc_fence_after();
-                issue_s<D, NT, KB>(tmem, q, qd + q * dd.qtile, dd.k0 + s * dd.stage);
+                issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + s * dd.stage);
                 sm100::tc_commit(&bars[C::bSFull + q]);
             }
             if (ok) sm100::tc_commit(&bars[C::bKEmpty + s]);
         }
-        if (ok) sm100::tc_commit(&bars[C::bQEmpty + qbuf]);  // this unit's Q is no longer read
+        if (ok) sm100::tc_commit(&bars[C::bQEmpty]);  // this unit's Q is no longer read
     }
     if (!ok) {
         record_error(kErrDeviceTimeout);
@@ -449,10 +433,8 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
         const Work w = decode<GQ>(p, unit);
         if (!unit_has_work<NT, GQ>(p, w)) continue;
         const int n = w.je - w.jb;  // blocks of this unit, counted from its first
-        const int qbuf = uq % C::kQBufs;
-        ok = sm100::mbar_wait(&bars[C::bQFull + qbuf], (uq / C::kQBufs) & 1, lim);
+        ok = sm100::mbar_wait(&bars[C::bQFull], uq & 1, lim);
         ++uq;
-        const uint64_t qd = dd.q0 + qbuf * dd.qbuf;
         sm100::tc_fence_after();
         for (int j = 0; ok && j <= n; ++j) {
             if (*abort_flag) {
@@ -478,13 +460,13 @@ __device__ void run_mma(const FwdParams &p, uint8_t *smem, uint64_t *bars, uint3
                     sm100::tc_commit(&bars[C::bPFree + q]);
                 }
                 if (j < n) {
-                    issue_s<D, NT, KB>(tmem, q, qd + q * dd.qtile, dd.k0 + (g % C::kStages) * dd.stage);
+                    issue_s<D, NT, KB>(tmem, q, dd.q0 + q * dd.qtile, dd.k0 + (g % C::kStages) * dd.stage);
                     sm100::tc_commit(&bars[C::bSFull + q]);
                 }
             }
             if (!ok) break;
             if (j < n) sm100::tc_commit(&bars[C::bKEmpty + g % C::kStages]);
-            if (j == n - 1) sm100::tc_commit(&bars[C::bQEmpty + qbuf]);
+            if (j == n - 1) sm100::tc_commit(&bars[C::bQEmpty]);
             if (j > 0) sm100::tc_commit(&bars[C::bVEmpty + (g - 1) % C::kStages]);
         }
         gb += n;
@@ -521,86 +503,23 @@ __device__ __forceinline__ float row_max(const float (&s)[KB]) {
     return sm100::max3(sm100::max3(mk[0], mk[1], mk[2]), sm100::max3(mk[3], mk[4], mk[5]), fmaxf(mk[6], mk[7]));
 }
 
-// Exponentials on the FMA pipe, to offload the special-function unit (MUFU),
-// which bounds the d = 64 softmax: every kPolyEvery-th pair of a thread's
-// exponentials in blocks without masked keys (0: none). Build option
-// NPA_EXP_POLY_EVERY.
-#ifndef NPA_EXP_POLY_EVERY
-#define NPA_EXP_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = NPA_EXP_POLY_EVERY;
-
-// Minimax coefficients (relative error on [-1/2, 1/2], found by the Remez
-// exchange; largest relative error 7.5e-5) of the cubic c0 + c1 f + c2 f^2 +
-// c3 f^3 that approximates 2^f.
-constexpr float kExp2C0 = 0.9999280571937561f, kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f, kExp2C3 = 0.0551716685295105f;
-
-// 2^x for a pair of finite arguments on the FMA pipe. x is clamped below at
-// -125 (the result is then about 2^-125, negligible next to the row sum,
-// which is at least 1), split as x = j + f with j = rint(x) - the float32
-// addition of 1.5 * 2^23 rounds to an integer held in the low mantissa bits -
-// and f = x - j in [-1/2, 1/2]; 2^f comes from the cubic above and 2^j is
-// added to its exponent field (j << 23; the constant's own bits shift out).
-__device__ __forceinline__ void exp2_fma_x2(uint64_t x2, float &p0, float &p1) {
-    float x0, x1;
-    sm100::unpack_f32x2(x2, x0, x1);
-    const uint64_t xc = sm100::pack_f32x2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = sm100::add_f32x2(xc, sm100::pack_f32x2(12582912.f, 12582912.f));
-    const uint64_t j = sm100::add_f32x2(t, sm100::pack_f32x2(-12582912.f, -12582912.f));
-    const uint64_t f = sm100::fma_f32x2(j, sm100::pack_f32x2(-1.f, -1.f), xc);
-    uint64_t q = sm100::fma_f32x2(sm100::pack_f32x2(kExp2C3, kExp2C3), f, sm100::pack_f32x2(kExp2C2, kExp2C2));
-    q = sm100::fma_f32x2(q, f, sm100::pack_f32x2(kExp2C1, kExp2C1));
-    q = sm100::fma_f32x2(q, f, sm100::pack_f32x2(kExp2C0, kExp2C0));
-    float q0, q1, t0, t1;
-    sm100::unpack_f32x2(q, q0, q1);
-    sm100::unpack_f32x2(t, t0, t1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
-// p = 2^(s*c - ref) for the scores of pairs [I0, I1): packed bf16 pairs
-// into pk, float32 partial sums into acc. POLY > 0: every POLY-th pair on the
-// FMA pipe (no -inf scores).
-template <int KB, int POLY, int I0, int I1>
-__device__ __forceinline__ void exp_range(const float (&s)[KB], uint64_t c2, uint64_t m2, uint32_t (&pk)[KB / 2],
-                                          uint64_t (&acc)[4]) {
-#pragma unroll
-    for (int i = I0; i < I1; ++i) {
-        const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
-        float p0, p1;
-        if (POLY > 0 && i % (POLY > 0 ? POLY : 1) == POLY - 1) {
-            exp2_fma_x2(x2, p0, p1);
-        } else {
-            float x0, x1;
-            sm100::unpack_f32x2(x2, x0, x1);
-            p0 = sm100::ex2_approx(x0);
-            p1 = sm100::ex2_approx(x1);
-        }
-        pk[i] = sm100::pack_bf16x2(p0, p1);
-        acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
-    }
-}
-
-// Hand-off point of the exponential unit's turn, in pairs before the end of a
-// thread's block (0: after the whole block is issued). Build option.
-#ifndef NPA_TURN_EARLY
-#define NPA_TURN_EARLY 0
-#endif
-
-// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum
-// returned; `handoff` runs after pair KB/2 - NPA_TURN_EARLY has been issued.
-template <int KB, int POLY, typename F>
-__device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2],
-                                           F &&handoff) {
+// p = 2^(s*c - ref) for KB scores: packed bf16 pairs into pk, float32 sum returned.
+template <int KB>
+__device__ __forceinline__ float exp_block(const float (&s)[KB], float c, float ref, uint32_t (&pk)[KB / 2]) {
     const float neg = (ref == -INFINITY) ? 0.f : -ref;
     const uint64_t c2 = sm100::pack_f32x2(c, c);
     const uint64_t m2 = sm100::pack_f32x2(neg, neg);
     uint64_t acc[4] = {0, 0, 0, 0};
-    constexpr int kSplit = KB / 2 - NPA_TURN_EARLY;
-    exp_range<KB, POLY, 0, kSplit>(s, c2, m2, pk, acc);
-    handoff();
-    exp_range<KB, POLY, kSplit, KB / 2>(s, c2, m2, pk, acc);
+#pragma unroll
+    for (int i = 0; i < KB / 2; ++i) {
+        const uint64_t x2 = sm100::fma_f32x2(sm100::pack_f32x2(s[2 * i], s[2 * i + 1]), c2, m2);
+        float x0, x1;
+        sm100::unpack_f32x2(x2, x0, x1);
+        const float p0 = sm100::ex2_approx(x0);
+        const float p1 = sm100::ex2_approx(x1);
+        pk[i] = sm100::pack_bf16x2(p0, p1);
+        acc[i & 3] = sm100::add_f32x2(acc[i & 3], sm100::pack_f32x2(p0, p1));
+    }
     float a0, a1, b0, b1, c0, c1, d0, d1;
     sm100::unpack_f32x2(acc[0], a0, a1);
     sm100::unpack_f32x2(acc[1], b0, b1);
@@ -665,12 +584,10 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         }
         // keys of this block outside its row segment or the window (or past
         // the last global token) get -inf
-        bool masked = false;  // some key of this block is outside its set
         if (j < w.n_win) {
             const int vc = w.wc1 - (w.wc0 + (btc << p.kc_log2));
             const int vr = bend - brow;
-            masked = vc < kc || vr < p.kr;
-            if (masked) {
+            if (vc < kc || vr < p.kr) {
 #pragma unroll
                 for (int i = 0; i < kC; ++i)
                     if ((i & (kc - 1)) >= vc || (i >> p.kc_log2) >= vr) s[i] = -INFINITY;
@@ -685,7 +602,6 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             }
         } else {
             const int vg = p.G - (j - w.n_win) * KB;
-            masked = vg < KB;
             if (vg < kC) {
 #pragma unroll
                 for (int i = 0; i < kC; ++i)
@@ -705,20 +621,15 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
             break;
         }
         uint32_t pk[kC / 2];
+        const float blk_sum = exp_block<kC>(s, sl2, R, pk);
         // pass the turn to the next warpgroup's warp on this sub-partition once
-        // the block's exponentials are issued (handing it over at 3/4 or 7/8
-        // of the block measured 16-17% slower)
-        auto handoff = [&]() {
-            if (C::kUseTurn) {
-                __syncwarp();
-                if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
-            }
-        };
-        float blk_sum;
-        if (kPolyEvery > 0 && C::kSeparateP && !masked)
-            blk_sum = exp_block<kC, (C::kSeparateP ? kPolyEvery : 0)>(s, sl2, R, pk, handoff);
-        else
-            blk_sum = exp_block<kC, 0>(s, sl2, R, pk, handoff);
+        // the whole block is issued (handing it over two, four or eight pairs
+        // before the end measured 14% slower, at 3/4 or 7/8 of the block
+        // 16-17% slower)
+        if (C::kUseTurn) {
+            __syncwarp();
+            if (lane0) sm100::mbar_arrive(&bars[C::bTurn + 4 * (q + 1 == NT ? 0 : q + 1) + warp_in_group]);
+        }
         const float alpha = (R == R_prev) ? 1.f : sm100::ex2_approx(R_prev - R);  // 0 on the first block
         if (C::kSeparateP && j > w.jb) {
             // PV_q(j-1) must be done before O is rescaled or P_q overwritten
@@ -856,10 +767,8 @@ __global__ void __launch_bounds__(KCfg<D, NT, KB>::kThreads, 1) npa_fwd_kernel(c
     const int warp = threadIdx.x >> 5;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < C::kQBufs; ++b) {
-            sm100::mbar_init(&bars[C::bQFull + b], 1);
-            sm100::mbar_init(&bars[C::bQEmpty + b], 1);
-        }
+        sm100::mbar_init(&bars[C::bQFull], 1);
+        sm100::mbar_init(&bars[C::bQEmpty], 1);
         for (int s = 0; s < C::kStages; ++s) {
             sm100::mbar_init(&bars[C::bKFull + s], 1);
             sm100::mbar_init(&bars[C::bKEmpty + s], 1);
