@@ -106,10 +106,7 @@ struct KCfg {
     static constexpr int kQTileBytes = kChunks * kQChunkBytes;
     static constexpr int kKVChunkBytes = KB * 128;         // KB key rows x 128 bytes
     static constexpr int kKVTileBytes = kChunks * kKVChunkBytes;
-#ifndef NPA_D64_STAGES
-#define NPA_D64_STAGES 4
-#endif
-    static constexpr int kStages = D == 128 ? 2 : NPA_D64_STAGES;
+    static constexpr int kStages = D == 128 ? 2 : 4;
     static constexpr int kThreads = 128 * (kSoftmaxWGs + 1);
     static constexpr int kCtlWarp = 4 * kSoftmaxWGs;       // first warp of the control warpgroup
     // registers per thread: at launch (the most __launch_bounds__ allows for
@@ -570,10 +567,7 @@ __device__ void run_softmax(const FwdParams &p, uint64_t *bars, uint32_t tmem, v
         float s[kC];
         {
             uint32_t sr[kC];
-            if constexpr (kC == 128)
-                sm100::tmem_ld128(tS, sr);
-            else
-                sm100::tmem_ld64(tS, sr);
+            sm100::tmem_ld128(tS, sr);
 #pragma unroll
             for (int i = 0; i < kC; ++i) s[i] = __uint_as_float(sr[i]);
         }

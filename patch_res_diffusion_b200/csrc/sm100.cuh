@@ -189,19 +189,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;\n"
-        : NPA_R8(0), NPA_R8(8), NPA_R8(16), NPA_R8(24), NPA_R8(32), NPA_R8(40), NPA_R8(48), NPA_R8(56)
-        : "r"(taddr)
-        : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
@@ -292,22 +279,6 @@ __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
 
 __device__ __forceinline__ void unpack_f32x2(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-// Two exponentials base 2 of a bf16x2 argument, bf16x2 result (flushes
-// subnormals; ex2(-inf) = +0).
-__device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
-    uint32_t y;
-    asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
-// acc + lo(v) + hi(v), the two bf16 halves widened exactly into float32 adds.
-__device__ __forceinline__ void add_bf16x2_to(float &acc_lo, float &acc_hi, uint32_t v) {
-    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}\n"
-        : "+f"(acc_lo), "+f"(acc_hi)
-        : "r"(v));
 }
 
 // Packs two floats into bf16x2 (round to nearest even); `lo` goes to the low half.
