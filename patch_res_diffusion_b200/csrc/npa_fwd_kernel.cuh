@@ -115,8 +115,8 @@ struct KCfg {
     // the control warpgroup gives registers back and the softmax warpgroups
     // take them
     static constexpr uint32_t kRegsLaunch = 168;
-    static constexpr uint32_t kRegsSoftmax = 216;
-    static constexpr uint32_t kRegsCtl = 72;
+    static constexpr uint32_t kRegsSoftmax = 208;
+    static constexpr uint32_t kRegsCtl = 88;  // the d = 128 MMA issuer spills below 88
     static_assert(kSoftmaxWGs * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
     static_assert(kThreads * kRegsLaunch <= 65536, "register file");
     static constexpr int kOffQ = 0;
