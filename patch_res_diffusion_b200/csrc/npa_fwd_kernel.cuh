@@ -114,9 +114,12 @@ struct KCfg {
     // since a split above the launch total would never complete), then after
     // the control warpgroup gives registers back and the softmax warpgroups
     // take them
+    // d = 128: the single MMA issuer spills below 88 control registers (and
+    // the kernel is 1.1% faster without); d = 64 spills in neither split and
+    // is 0.3-0.5% faster with the larger softmax share
     static constexpr uint32_t kRegsLaunch = 168;
-    static constexpr uint32_t kRegsSoftmax = 208;
-    static constexpr uint32_t kRegsCtl = 88;  // the d = 128 MMA issuer spills below 88
+    static constexpr uint32_t kRegsSoftmax = D == 64 ? 216 : 208;
+    static constexpr uint32_t kRegsCtl = D == 64 ? 72 : 88;
     static_assert(kSoftmaxWGs * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
     static_assert(kThreads * kRegsLaunch <= 65536, "register file");
     static constexpr int kOffQ = 0;
