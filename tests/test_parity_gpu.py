@@ -209,6 +209,49 @@ def test_bitwise_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("kind", ["npa_4096", "flux_edge_geometry", "pcpp_8x16", "pcpp_stale", "global_query_split",
+                                  "multidiffusion"])
+def test_bitwise_deterministic_every_path(kind):
+    """Two calls on the same inputs give the same bits on every path: the
+    persistent schedule, the per-CTA unit lists (head by head or by class)
+    and the split combines use no atomics and no order that depends on
+    timing."""
+    import patch_res_diffusion_b200 as npa
+    rng = np.random.default_rng(21)
+    r = lambda *shape: to_device(f64_to_bf16_bits(rng.standard_normal(shape)))
+    if kind == "npa_4096":
+        w = PRESETS["npa_sdxl_4096"]
+        q, k, v = (r(w.B, w.heads, w.H * w.W, w.d) for _ in range(3))
+        call = lambda: npa.npa_attention(q, k, v, w.H, w.W, w.patch, w.margin)
+    elif kind == "flux_edge_geometry":
+        H, W = 96, 80
+        q, k, v, gk, gv = r(1, 4, H * W, 128), r(1, 4, H * W, 128), r(1, 4, H * W, 128), r(1, 4, 70, 128), \
+            r(1, 4, 70, 128)
+        call = lambda: npa.npa_attention(q, k, v, H, W, 32, 16, gk, gv)
+    elif kind == "pcpp_8x16":
+        w = PRESETS["pcpp_8x16_p0.8"]
+        q, k, v = (r(w.B, w.heads, w.H * w.W, w.d) for _ in range(3))
+        call = lambda: npa.pcpp_attention(q, k, v, w.H, w.W, w.n_strips, w.p)
+    elif kind == "pcpp_stale":
+        H, W = 64, 96
+        q, k, v, ks, vs = (r(2, 3, H * W, 64) for _ in range(5))
+        call = lambda: npa.pcpp_attention_stale(q, k, v, ks, vs, H, W, 4, 0.3)
+    elif kind == "global_query_split":
+        H, W = 64, 64
+        q, gk, gv = r(1, 6, 300, 128), r(1, 6, 300, 128), r(1, 6, 300, 128)
+        k, v = r(1, 6, H * W, 128), r(1, 6, H * W, 128)
+        call = lambda: npa.global_query_attention(q, k, v, gk, gv, H, W, split=True)
+    else:
+        H, W = 72, 64
+        q, k, v = (r(1, 3, H * W, 64) for _ in range(3))
+        call = lambda: npa.multidiffusion_attention(q, k, v, H, W, 16, 6)
+    a = call()
+    b = call()
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert npa.npa_device_status() == npa.NPA_OK
+
+
 def test_side_stream_ordering():
     w = SMALL[2]
     inp = make_inputs(w)
