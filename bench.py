@@ -85,12 +85,23 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments, trailing spaces or blank lines (string
+    literals are kept as they are)."""
+    import re
+    pattern = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^"\\])*"', re.S)
+    src = pattern.sub(lambda m: m.group(0) if m.group(0).startswith('"') else "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources (csrc/), comments and layout excluded: the
+    recorded ncu counters apply while the code itself is unchanged."""
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "patch_res_diffusion_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+        with open(f, encoding="utf-8") as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(_strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -13,8 +13,8 @@
 // Work unit = (batch*head, patch, group of tiles_per_unit 128-row query
 // tiles); a persistent CTA walks the units blockIdx.x, blockIdx.x + gridDim.x,
 // ... A query tile is a box of qr patch rows x qc patch columns (qr*qc <=
-// 128); a key/value block is a box of kr rows x kc columns (kr*kc = kb, 64 or
-// 128 keys) inside the window, followed by ceil(G/kb) blocks of global
+// 128); a key/value block is a box of kr rows x kc columns (kr*kc = kb = 128
+// keys) inside the window, followed by ceil(G/kb) blocks of global
 // tokens. Every quantity is recomputed from the unit index with integer
 // arithmetic; the only table is the host-built patch order.
 #pragma once
@@ -51,9 +51,9 @@ struct FwdParams {
     int Ph, Pw, mh, mw;
     int nPh, nPw;                    // patches along rows / columns
     int qc, qr, tiles_c, tiles_r;    // query tile box and tiles per patch
-    int kb;                          // keys per key block (64 or 128)
+    int kb;                          // keys per key block (128)
     int kc_log2, kr;                 // key block box: (1 << kc_log2) columns x kr rows
-    int tiles_per_unit;              // query tiles per work unit (2 or 3)
+    int tiles_per_unit;              // query tiles per work unit (2)
     int n_qblocks;                   // query-tile groups per patch
     float scale_log2;                // log2(e) / sqrt(d)
     unsigned long long wait_limit_ns;
