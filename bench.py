@@ -187,9 +187,10 @@ def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
         pairs = sum(key_count(int(t)) + w.G * (md_cover(w, int(t)) if w.geometry == "md" else 1)
                     for t in qs[:, 2])
         t0 = time.perf_counter()
-        fn(inp["q"], inp["k"], inp["v"], gk=inp.get("gk"), gv=inp.get("gv"), G=w.G, B=w.B, heads=w.heads,
-           H=w.H, W=w.W, d=w.d, queries=qs, **geom)
+        out = fn(inp["q"], inp["k"], inp["v"], gk=inp.get("gk"), gv=inp.get("gv"), G=w.G, B=w.B, heads=w.heads,
+                 H=w.H, W=w.W, d=w.d, queries=qs, **geom)
         dt = time.perf_counter() - t0
+        last_sample = (qs, out)
         total_q += n
         total_pairs += pairs
         total_t += dt
@@ -202,6 +203,7 @@ def oracle_rate(w: Workload, inp: dict, seconds: float) -> dict:
         "kind": "oracle",
         "sample": f"{total_q} uniformly drawn (b, h, query) rows of {w.name}, float64, {total_t:.1f} s",
         "seconds": total_t,
+        "last_sample": last_sample,
     }
 
 
@@ -500,6 +502,24 @@ def per_config_entry(prep, res: dict, pk: dict) -> dict:
     }
 
 
+def sample_parity(w: Workload, o, qs: np.ndarray, ref: np.ndarray) -> dict:
+    """The timed call's output against the float64 oracle on the rows the CPU
+    baseline computed (the same seeded inputs): max and mean absolute
+    difference and relative L2, with the gates the tests use."""
+    import torch
+    rows = w.G if w.geometry == "gq" else w.H * w.W
+    flat = o.reshape(-1, w.d)
+    idx = torch.from_numpy((qs[:, 0].astype(np.int64) * w.heads + qs[:, 1]) * rows + qs[:, 2]).to(o.device)
+    got = flat.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+    diff = np.abs(got - ref)
+    m = {"rows": int(len(qs)), "max_abs": float(diff.max()), "mean_abs": float(diff.mean()),
+         "rel_l2": float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))}
+    m["within_gates"] = bool(np.isfinite(got).all() and m["max_abs"] <= 2e-2 and m["mean_abs"] <= 2e-3
+                             and m["rel_l2"] <= 1e-2)
+    m["gates"] = "max |d| <= 2e-2, mean |d| <= 2e-3, relative L2 <= 1e-2 against the float64 oracle"
+    return m
+
+
 # The other target workloads reported beside the headline one.
 PER_CONFIG = ["tiny_npa", "pcpp_4x32_p0.3", "pcpp_8x16_p0.8", "npa_sdxl_2048", "npa_flux_4096"]
 
@@ -621,9 +641,12 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "hbm_min_bytes_per_launch": bytes_io,
     }
     cpu = None
+    parity = None
     if not args.no_cpu_baseline and world == 1:
         cpu = oracle_rate(w, inp, args.cpu_seconds)
         cpu.pop("seconds", None)
+        qs, ref = cpu.pop("last_sample")
+        parity = sample_parity(w, o, qs, ref)
     cfg = describe(w)
     cfg["parallelism"] = f"replicas x{world}" if world > 1 else "single GPU"
     cfg["l2"] = ("flushed (256 MB write) between launches; value from per-launch events" if flush is not None
@@ -649,6 +672,8 @@ def run_ours(args, w: Workload, rank: int, world: int, local_rank: int) -> None:
         "gpu_launches": args.steps * prep.launches,
         "kernel_ms": {"median": statistics.median(kernel_ms), "best": min(kernel_ms)},
     }
+    if parity is not None:
+        line["parity"] = parity
     if per_config is not None:
         line["per_config"] = per_config
     print(json.dumps(line), flush=True)

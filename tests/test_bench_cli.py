@@ -59,3 +59,29 @@ def test_max_over_ranks_and_whole_job_rate_gloo(tmp_path, world):
     for got_ms, rate in results:
         assert got_ms == slowest
         assert rate == world * 1e12 * 10 / (slowest * 1e-3)
+
+
+def test_sample_parity_indexes_the_sampled_rows():
+    """bench.sample_parity gathers output rows (b, h, t) of a [B, heads, N, d]
+    tensor and compares them with oracle rows; checked on the CPU with the
+    oracle's own full output rounded to bf16 (within the gates) and with one
+    sampled row planted wrong (outside them)."""
+    import numpy as np
+    import torch
+    import bench
+    import oracle
+    from workloads import Workload, make_inputs
+    w = Workload("cpu_tiny", "npa", B=2, heads=3, H=8, W=6, d=64, patch=4, margin=2)
+    inp = make_inputs(w)
+    full = oracle.npa_attention(inp["q"], inp["k"], inp["v"], B=w.B, heads=w.heads, H=w.H, W=w.W, d=w.d,
+                                patch=w.patch, margin=w.margin)
+    o = torch.from_numpy(full).to(torch.bfloat16)
+    rng = np.random.default_rng(0)
+    qs = np.stack([rng.integers(w.B, size=40), rng.integers(w.heads, size=40), rng.integers(w.H * w.W, size=40)],
+                  1).astype(np.int32)
+    ref = np.stack([full[b, h, t] for b, h, t in qs])
+    m = bench.sample_parity(w, o, qs, ref)
+    assert m["rows"] == 40 and m["within_gates"] and m["rel_l2"] < 1e-2
+    b, h, t = qs[7]
+    o[b, h, t] += 0.5
+    assert not bench.sample_parity(w, o, qs, ref)["within_gates"]
