@@ -252,6 +252,29 @@ def test_bitwise_deterministic_every_path(kind):
     assert npa.npa_device_status() == npa.NPA_OK
 
 
+def test_schedule_cache_eviction_keeps_results():
+    """The host keeps the per-CTA unit lists of the last 8 geometries. Running
+    10 geometries (PCPP and NPA, class split and ragged) and then the first
+    ones again - rebuilt after eviction - gives the same bits, and the first
+    pass matches the oracle."""
+    import patch_res_diffusion_b200 as npa
+    geoms = [Workload(f"cache_{i}", "pcpp" if i % 2 else "npa", B=1, heads=1 + i % 3, H=32 + 8 * (i % 4),
+                      W=40 + 8 * (i % 3), d=64, patch=8 + 4 * (i % 3), margin=2 + i % 5, n_strips=4, p=0.25 + 0.1 * (i % 3))
+             for i in range(10)]
+    first = []
+    for w in geoms:
+        inp = make_inputs(w)
+        o = run_gpu(w, inp)
+        m = compare(to_f64(o), run_oracle(w, inp))
+        assert passes(m), (w.name, m)
+        first.append((w, inp, o))
+    for w, inp, o in first[:4]:
+        again = run_gpu(w, inp)
+        torch.cuda.synchronize()
+        assert torch.equal(again.view(torch.int16), o.view(torch.int16)), w.name
+    assert npa.npa_device_status() == npa.NPA_OK
+
+
 def test_side_stream_ordering():
     w = SMALL[2]
     inp = make_inputs(w)
