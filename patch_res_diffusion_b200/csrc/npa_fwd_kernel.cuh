@@ -109,14 +109,13 @@ struct KCfg {
     static constexpr int kStages = D == 128 ? 2 : 4;
     static constexpr int kThreads = 128 * (kSoftmaxWGs + 1);
     static constexpr int kCtlWarp = 4 * kSoftmaxWGs;       // first warp of the control warpgroup
-    // registers per thread: at launch (the most __launch_bounds__ allows for
+    // Registers per thread: at launch (the most __launch_bounds__ allows for
     // kThreads; the host checks the compiled count before the first launch,
     // since a split above the launch total would never complete), then after
     // the control warpgroup gives registers back and the softmax warpgroups
-    // take them
-    // d = 128: the single MMA issuer spills below 88 control registers (and
-    // the kernel is 1.1% faster without); d = 64 spills in neither split and
-    // is 0.3-0.5% faster with the larger softmax share
+    // take them. At d = 128 the single MMA issuer spills below 88 control
+    // registers (and the kernel is 1.1% faster without); d = 64 spills in
+    // neither split and is 0.3-0.5% faster with the larger softmax share.
     static constexpr uint32_t kRegsLaunch = 168;
     static constexpr uint32_t kRegsSoftmax = D == 64 ? 216 : 208;
     static constexpr uint32_t kRegsCtl = D == 64 ? 72 : 88;
