@@ -345,3 +345,37 @@ def test_cuda_graph_replay(kind):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), eager2.view(torch.int16))
     assert not torch.equal(eager.view(torch.int16), eager2.view(torch.int16))
+
+
+def _random_geometries(n, seed=2024):
+    """Seeded small geometries: NPA and PCPP, d 64 or 128, ragged grids and
+    patches, margins from 0 past the patch, optional global tokens."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        d = int(rng.choice([64, 128]))
+        B, heads = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+        H, W = int(rng.integers(3, 70)), int(rng.integers(3, 90))
+        G = int(rng.choice([0, 0, int(rng.integers(1, 200))]))
+        if rng.random() < 0.5:
+            patch = int(rng.integers(1, max(2, min(H, W))))
+            margin = int(rng.integers(0, patch + 6))
+            out.append(Workload(f"rand_npa_{i}", "npa", B=B, heads=heads, H=H, W=W, d=d, patch=patch, margin=margin,
+                                G=G, seed=i))
+        else:
+            divisors = [s for s in range(1, H + 1) if H % s == 0]
+            n_strips = int(rng.choice(divisors))
+            p = float(rng.choice([0.0, 0.1, 0.3, 0.5, 0.8, 1.0]))
+            out.append(Workload(f"rand_pcpp_{i}", "pcpp", B=B, heads=heads, H=H, W=W, d=d, n_strips=n_strips, p=p,
+                                G=G, seed=i))
+    return out
+
+
+@pytest.mark.parametrize("w", _random_geometries(24), ids=lambda w: w.name)
+def test_random_geometries_parity(w):
+    """Seeded random small geometries through the whole path (unit numbering,
+    per-CTA lists and their cache, masks, global tokens) against the oracle."""
+    inp = make_inputs(w)
+    m = compare(to_f64(run_gpu(w, inp)), run_oracle(w, inp))
+    log_metrics("random " + w.name, m)
+    assert passes(m), (w, m)
