@@ -71,3 +71,18 @@ def test_global_query_flux_shape_every_row(split):
     m = compare(got, _FLUX_REF["ref"])
     log_metrics(f"global query FLUX split={split} (every row)", m)
     assert passes(m), m
+
+
+@pytest.mark.parametrize("i", range(8))
+def test_random_global_query_shapes(i):
+    """Seeded random text-query shapes, split and unsplit, against the oracle."""
+    rng = np.random.default_rng(300 + i)
+    B, heads = int(rng.integers(1, 3)), int(rng.integers(1, 6))
+    H, W, d, G = int(rng.integers(1, 48)), int(rng.integers(1, 48)), int(rng.choice([64, 128])), int(rng.integers(1, 400))
+    inp = make(B, heads, H, W, d, G, 400 + i)
+    ref = oracle.global_query_attention(inp["gq"], inp["k"], inp["v"], inp["gk"], inp["gv"], B=B, heads=heads, H=H,
+                                        W=W, d=d, G=G)
+    for split in (False, True):
+        m = compare(to_f64(gpu(inp, H, W, split)), ref)
+        log_metrics(f"random global query {B}x{heads} {H}x{W} d{d} G{G} split={split}", m)
+        assert passes(m), (B, heads, H, W, d, G, split, m)

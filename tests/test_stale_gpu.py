@@ -120,3 +120,38 @@ def test_stale_full_workload_every_row(name):
     m = compare(to_f64(run_gpu(w, inp)), run_oracle(w, inp))
     log_metrics("stale " + name + " (every row)", m)
     assert passes(m), m
+
+
+def _random_stale(n, seed=77):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        H = int(rng.integers(4, 64))
+        divisors = [s for s in range(1, H + 1) if H % s == 0 and H // s >= 1]
+        n_strips = int(rng.choice(divisors))
+        begin = int(rng.integers(0, n_strips))
+        count = int(rng.integers(1, n_strips - begin + 1))
+        w = Workload(f"rand_stale_{i}", "pcpp", B=int(rng.integers(1, 3)), heads=int(rng.integers(1, 3)), H=H,
+                     W=int(rng.integers(3, 100)), d=int(rng.choice([64, 128])), n_strips=n_strips,
+                     p=float(rng.choice([0.0, 0.2, 0.5, 1.0])), G=int(rng.choice([0, int(rng.integers(1, 90))])),
+                     seed=i)
+        out.append((w, (begin, count)))
+    return out
+
+
+@pytest.mark.parametrize("case", _random_stale(12), ids=lambda c: c[0].name)
+def test_random_stale_strip_ranges(case):
+    """Seeded random two-source geometries and strip ranges: the computed
+    strips match the oracle, the others are left untouched."""
+    w, (begin, count) = case
+    inp = stale_inputs(w)
+    got = to_f64(run_gpu(w, inp, strips=(begin, count)))
+    ref = run_oracle(w, inp)
+    s = w.H // w.n_strips * w.W
+    sel = slice(begin * s, (begin + count) * s)
+    m = compare(got[:, :, sel], ref[:, :, sel])
+    log_metrics("random " + w.name, m)
+    assert passes(m), (w, begin, count, m)
+    rest = np.ones(w.H * w.W, dtype=bool)
+    rest[sel] = False
+    assert np.isnan(got[:, :, rest]).all()
