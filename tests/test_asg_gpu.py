@@ -80,3 +80,17 @@ def test_in_place_and_special_cases():
     full = npa.asg_combine(to_device(eps), to_device(ref), to_device(ones), 1.0)
     torch.cuda.synchronize()
     assert np.array_equal(gpu_bits(full), np.broadcast_to(ref[None], eps.shape))   # full pull: the reference
+
+
+@pytest.mark.parametrize("i", range(6))
+def test_random_shapes(i):
+    """Seeded random shapes (ragged pixel counts included) and weights."""
+    import patch_res_diffusion_b200 as npa
+    rng = np.random.default_rng(500 + i)
+    n, B, C = int(rng.integers(1, 6)), int(rng.integers(1, 4)), int(rng.integers(1, 6))
+    S = int(rng.integers(max(1, 2000 // (n * B * C)), 5000))
+    w = float(rng.uniform(-2.0, 3.0))
+    eps, ref, m = make(n, B, C, S, seed=600 + i)
+    out = npa.asg_combine(to_device(eps), to_device(ref), to_device(m), w)
+    torch.cuda.synchronize()
+    check(gpu_bits(out), oracle.asg_guidance_combine(eps, ref, m, w), eps, ref, m, w)

@@ -94,3 +94,25 @@ def test_sdxl_shapes_sampled(shape):
     m = compare(got, ref(w, inp, queries=qs))
     log_metrics(f"multidiffusion {shape} sampled", m)
     assert passes(m), m
+
+
+def _random_md(n, seed=55):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        H, W = int(rng.integers(2, 48)), int(rng.integers(2, 48))
+        patch = int(rng.integers(1, max(2, min(H, W) + 1)))
+        out.append(Workload(f"rand_md_{i}", "npa", B=int(rng.integers(1, 3)), heads=int(rng.integers(1, 3)), H=H, W=W,
+                            d=int(rng.choice([64, 128])), patch=patch, margin=int(rng.integers(0, patch + 4)),
+                            G=int(rng.choice([0, int(rng.integers(1, 40))])), seed=i))
+    return out
+
+
+@pytest.mark.parametrize("w", _random_md(10), ids=lambda w: w.name)
+def test_random_geometries_full_parity(w):
+    """Seeded random small geometries of the comparator, every row against the oracle."""
+    inp = make_inputs(w)
+    m = compare(to_f64(gpu(w, inp)), ref(w, inp))
+    log_metrics(f"random multidiffusion {w.name}", m)
+    assert passes(m), (w, m)
