@@ -45,9 +45,12 @@
  * entry points allocate no device memory; the library's device state is one
  * status word per device (see npa_device_status) and the fixed scratch array
  * of npa_global_query_attention_fwd_noalloc. Host-side state is
- * limited to per-device capability checks, kernel attributes and that array's
- * device address, set up under a lock on first use, so the entry points are
- * safe to call from several host threads.
+ * limited to per-device capability checks, kernel attributes, that array's
+ * device address (set up under a lock on first use) and a small cache of the
+ * per-CTA work lists of recently launched geometries (under its own lock), so
+ * the entry points are safe to call from several host threads. The first call
+ * of a new geometry builds its work lists on the host (0.1-0.5 ms); later
+ * calls take them from the cache.
  *
  * CUDA graphs: after a first call on a device (which checks the device and
  * sets kernel attributes), npa_attention_fwd, pcpp_attention_fwd,
